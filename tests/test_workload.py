@@ -1,0 +1,74 @@
+"""Host-side checks of the seeded synthetic workloads (no GPU)."""
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_global_b200 import workload as W
+from oracle import ress_oracle as O
+
+
+def test_special_token_tail_blocks():
+    # 8 views: 10992 tokens, 40 specials -> only the last block (112 tokens) holds them
+    assert W.special_tail_blocks(8 * 1374, 40) == [85]
+    assert W.special_tail_blocks(32 * 1374, 160) == [342, 343]
+    assert W.special_tail_blocks(100 * 1374, 500) == [1069, 1070, 1071, 1072, 1073]
+    assert W.special_tail_blocks(64 * 1374, 320) == [684, 685, 686]
+    assert W.num_blocks(100 * 1374) == 1074
+
+
+def test_uniform_budgets():
+    assert W.uniform_budget(0.5, 85) == 43
+    assert W.uniform_budget(0.75, 342) == 86
+    assert W.uniform_budget(0.9, 1069) == 107
+    assert [W.uniform_budget(s, 684) for s in W.SWEEP_SPARSITIES] == [684, 513, 342, 171, 68]
+    assert W.uniform_budget(0.99, 8) == 2          # two-block floor
+    assert W.uniform_budget(0.5, 1) == 1
+
+
+def test_allocation_respects_total_cap_floor():
+    rng = np.random.default_rng(0)
+    for _ in range(50):
+        w = rng.dirichlet(np.ones(16)).tolist()
+        out = W.allocate_budgets(w, 16 * 107, cap=1069, floor=2)
+        assert sum(out) == 16 * 107
+        assert min(out) >= 2 and max(out) <= 1069
+    out = W.allocate_budgets([0.97] + [0.002] * 15, 16 * 107, cap=1069, floor=2)
+    assert out[0] == 1069 and sum(out) == 16 * 107
+    out = W.allocate_budgets([0.25] * 4, 40, cap=12, floor=2)
+    assert out == [10, 10, 10, 10]
+
+
+def test_tiny_workload_shapes_and_layout():
+    wl = W.make_workload(1)
+    assert wl.q.shape == (1, 4, 1024, 64) and wl.q.dtype == torch.bfloat16
+    assert wl.budgets == [4, 4, 4, 4] and wl.rounds == 2
+    assert int(wl.keep_k.sum()) == 0 and int(wl.dense_q.sum()) == 0
+    wl2 = W.make_workload(1)
+    assert torch.equal(wl.q, wl2.q) and torch.equal(wl.w_o, wl2.w_o)
+
+
+def test_vggt_workload_small_variant():
+    wl = W.make_workload(2, heads=2, views=2)
+    n = 2 * 1374
+    assert wl.q.shape == (1, 2, n, 64)
+    assert wl.keep_k.tolist()[-1] == 1 and wl.dense_q.tolist()[-1] == 1
+    q = wl.q.float()
+    # special tokens (tail) carry the high norm
+    assert q[0, :, -10:].norm(dim=-1).mean() > 2 * q[0, :, :100].norm(dim=-1).mean()
+
+
+def test_near_duplicate_views_cosine():
+    wl = W.make_workload(4, heads=2, views=6)
+    assert len(wl.extras["near_duplicate_views"]) == 5
+    assert wl.extras["near_duplicate_min_cos"] >= 0.9
+    assert sum(wl.budgets) == 2 * W.uniform_budget(0.9, wl.nb - 1) or sum(wl.budgets) >= 2 * 2
+
+
+def test_oracle_layer_runs_on_tiny_case():
+    wl = W.make_workload(1)
+    for method in (O.MASS, O.DRIFT, O.RANDOM):
+        res = O.layer(wl.q, wl.k, wl.v, wl.w_o, method, wl.budgets, rounds=2, seed=wl.select_seed,
+                      rows=[(0, h, i) for h in range(4) for i in range(8)])
+        assert all(len(v) == 4 for v in res["kept"].values())
+        o, lse = res["attn"][(0, 1, 3)]
+        assert o.shape == (128, 64) and np.isfinite(o).all()
