@@ -1,0 +1,56 @@
+// Host-side launchers shared between the translation units of libress.so.  Arguments
+// have been validated by the C entry points (ress_api.cu) before any of these is called.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/ress.h"
+
+namespace ress {
+
+struct Dims {
+  int B, H, N, nb;
+  long long BH() const { return 1ll * B * H; }
+};
+
+cudaError_t launch_head_gram(int H, int d_model, const float *w_o, float *gram, cudaStream_t st);
+
+cudaError_t launch_pool(const Dims &d, const void *q, const void *k, const void *v, float *qp,
+                        float *kp, float *vp, cudaStream_t st);
+
+cudaError_t launch_block_scores(const Dims &d, const float *qp, const float *kp, const float *vp,
+                                float scale, float *P, float *vbar, cudaStream_t st);
+
+size_t drift_workspace_bytes(const Dims &d);
+cudaError_t launch_drift(const Dims &d, const float *P, const float *vp, const float *vbar,
+                         const float *gram, float *s, void *ws, cudaStream_t st);
+
+struct SelectLaunch {
+  int method, rounds;
+  float rho, eps;
+  uint64_t seed;
+  const int32_t *budgets;  // host [H]
+  const uint8_t *keep_k, *dense_q;
+  const float *P, *s, *vp, *vbar, *gram;
+  int32_t *kv_idx, *kv_cnt;
+  uint8_t *mask;
+  int32_t *dev_err;
+};
+cudaError_t launch_select(const Dims &d, const SelectLaunch &a, cudaStream_t st);
+
+cudaError_t launch_schedule(const Dims &d, const int32_t *kv_cnt, int32_t *order, cudaStream_t st);
+
+struct AttnLaunch {
+  const void *q, *k, *v;
+  const int32_t *kv_idx, *kv_cnt, *order;
+  float scale;
+  void *out;
+  float *lse;
+  int32_t *dev_err;
+};
+// Returns cudaErrorNotSupported if the driver cannot encode tensor maps.
+cudaError_t launch_attn(const Dims &d, const AttnLaunch &a, cudaStream_t st);
+
+}  // namespace ress

@@ -1,0 +1,104 @@
+"""One global-attention layer through libress: device buffers (torch) + the C-ABI calls.
+
+    layer = SparseGlobalAttention(batch, heads, seq_len)
+    layer.load_output_projection(w_o)          # M_h, once per layer
+    out = layer.forward(q, k, v, method=..., budgets=[...], keep_k=..., dense_q=...)
+
+Every step runs in the library's kernels; this class only owns the buffers and orders
+the calls on one stream: pool -> block map -> (drift) -> select -> schedule -> attention.
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional, Sequence
+
+import torch
+
+from . import ress as R
+
+
+class SparseGlobalAttention:
+    def __init__(self, batch: int, heads: int, seq_len: int, device="cuda", with_mask: bool = False):
+        self.B, self.H, self.N = batch, heads, seq_len
+        self.nb = (seq_len + R.BLOCK - 1) // R.BLOCK
+        self.shape = R.make_shape(batch, heads, seq_len)
+        self.device = torch.device(device)
+        B, H, nb, N = batch, heads, self.nb, seq_len
+        f32 = dict(device=self.device, dtype=torch.float32)
+        i32 = dict(device=self.device, dtype=torch.int32)
+        self.q_pool = torch.empty(B, H, nb, 64, **f32)
+        self.k_pool = torch.empty(B, H, nb, 64, **f32)
+        self.v_pool = torch.empty(B, H, nb, 64, **f32)
+        self.P = torch.empty(B, H, nb, nb, **f32)
+        self.v_bar = torch.empty(B, H, nb, 64, **f32)
+        self.s = torch.empty(B, H, nb, nb, **f32)
+        self.workspace = torch.empty(max(R.ress_drift_workspace_bytes(self.shape), 16),
+                                     device=self.device, dtype=torch.uint8)
+        self.kv_idx = torch.empty(B, H, nb, nb, **i32)
+        self.kv_cnt = torch.empty(B, H, nb, **i32)
+        self.order = torch.empty(B * H * nb, **i32)
+        self.mask = torch.empty(B, H, nb, nb, device=self.device, dtype=torch.uint8) if with_mask else None
+        self.out = torch.empty(B, H, N, 64, device=self.device, dtype=torch.bfloat16)
+        self.lse = torch.empty(B, H, N, **f32)
+        self.dev_err = torch.zeros(4, **i32)
+        self.gram = torch.empty(H, 64, 64, **f32)
+        self.scale = 1.0 / math.sqrt(64)
+
+    def load_output_projection(self, w_o: torch.Tensor, stream=None):
+        """M_h = W_O^h^T W_O^h for every head (ReSS Eq. 8), computed once per layer."""
+        R.ress_head_gram(self.shape, w_o.contiguous().float(), self.gram, stream)
+
+    # ------------------------------------------------------------------ the path
+    def scores(self, q, k, v, stream=None):
+        R.ress_pool_blocks(self.shape, q, k, v, self.q_pool, self.k_pool, self.v_pool, stream)
+        R.ress_block_scores(self.shape, self.q_pool, self.k_pool, self.v_pool, self.scale, self.P,
+                            self.v_bar, stream)
+
+    def drift(self, stream=None):
+        R.ress_drift_scores(self.shape, self.P, self.v_pool, self.v_bar, self.gram, self.s,
+                            self.workspace, stream)
+
+    def select(self, method: int, budgets: Sequence[int], keep_k=None, dense_q=None, rounds: int = 0,
+               rho: float = 0.5, eps: float = 1e-4, seed: int = 0, stream=None):
+        params = R.select_params(method, budgets, keep_k, dense_q, rounds, rho, eps, seed)
+        drift = method == R.SELECT_DRIFT
+        R.ress_select_blocks(self.shape, params, self.P, self.s if drift else None,
+                             self.v_pool if drift else None, self.v_bar if drift else None,
+                             self.gram if drift else None, self.kv_idx, self.kv_cnt, self.mask,
+                             self.dev_err, stream)
+
+    def attend(self, q, k, v, stream=None, schedule: bool = True):
+        if schedule:
+            R.ress_attn_schedule(self.shape, self.kv_cnt, self.order, stream)
+        R.ress_block_sparse_attn(self.shape, q, k, v, self.kv_idx, self.kv_cnt,
+                                 self.order if schedule else None, self.scale, self.out, self.lse,
+                                 self.dev_err, stream)
+
+    def forward(self, q, k, v, method: int, budgets: Sequence[int], keep_k=None, dense_q=None,
+                rounds: int = 0, rho: float = 0.5, eps: float = 1e-4, seed: int = 0, stream=None):
+        self.scores(q, k, v, stream)
+        if method == R.SELECT_DRIFT:
+            self.drift(stream)
+        self.select(method, budgets, keep_k, dense_q, rounds, rho, eps, seed, stream)
+        self.attend(q, k, v, stream)
+        return self.out
+
+    def kernel_launches(self, method: int) -> int:
+        """Kernels one forward() launches: pool, scores, [drift prep + drift], select,
+        schedule, attention."""
+        return 7 if method == R.SELECT_DRIFT else 5
+
+    def device_error(self) -> int:
+        return int(self.dev_err[0].item())
+
+    def kept_lists(self):
+        """{(b,h,i): ascending kept key blocks} from the device kv list (host copy)."""
+        idx = self.kv_idx.cpu()
+        cnt = self.kv_cnt.cpu()
+        out = {}
+        for b in range(self.B):
+            for h in range(self.H):
+                for i in range(self.nb):
+                    c = int(cnt[b, h, i])
+                    out[(b, h, i)] = idx[b, h, i, :c].tolist()
+        return out

@@ -1,0 +1,164 @@
+"""Helpers shared by the GPU parity tests: run the CUDA path through the C ABI, run the
+oracle on the same inputs, and compare with the tolerances below.
+
+Tolerances (fp32 intermediates, bf16 attention output):
+    pooled means, P, vbar : |gpu - oracle| <= 1e-4 |oracle| + floor  (summation order only)
+    drift s               : |gpu - oracle| <= 1e-4 |s| + P sqrt(1e-6 (a + 2|b| + c)), the
+                            cancellation bound of the Eq. 9 expansion a - 2b + c evaluated
+                            in fp32 (a = vbar^T M vbar, b = vbar^T M V_j, c = V_j^T M V_j)
+    kept-block lists      : identical on every row whose oracle decision margin exceeds
+                            1e-3 (relative); at least 99.9 % of all mask bits equal
+    attention             : max |gpu - oracle| <= 2e-2 and relative L2 <= 1e-2, the oracle
+                            run in fp32 on the GPU's own kept lists; LSE within 1e-3 + 1e-4|lse|
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+from block_sparse_global_b200 import build as B
+from block_sparse_global_b200 import ress as R
+from block_sparse_global_b200.pipeline import SparseGlobalAttention
+from oracle import ress_oracle as O
+
+MARGIN = 1e-3
+
+
+def ensure_built():
+    B.build()
+    R.load()
+
+
+def run_gpu(wl, method=None, rounds=None, with_mask=True, seed=None):
+    ensure_built()
+    dev = torch.device("cuda")
+    method = wl.method if method is None else method
+    rounds = wl.rounds if rounds is None else rounds
+    if method != O.DRIFT:
+        rounds = 0
+    q, k, v = wl.q.to(dev), wl.k.to(dev), wl.v.to(dev)
+    b, h, n, _ = q.shape
+    layer = SparseGlobalAttention(b, h, n, device=dev, with_mask=with_mask)
+    layer.load_output_projection(wl.w_o.to(dev))
+    layer.forward(q, k, v, method, wl.budgets, wl.keep_k.to(dev), wl.dense_q.to(dev), rounds,
+                  wl.rho, wl.eps, wl.select_seed if seed is None else seed)
+    torch.cuda.synchronize()
+    assert layer.device_error() == 0, f"device error {layer.device_error()}"
+    return layer
+
+
+class OracleLayer:
+    """Oracle intermediates for one workload (pooled tensors and P for every row)."""
+
+    def __init__(self, wl):
+        self.q = O.to_numpy_f32(wl.q)
+        self.k = O.to_numpy_f32(wl.k)
+        self.v = O.to_numpy_f32(wl.v)
+        self.B, self.H, self.N, _ = self.q.shape
+        self.scale = 1.0 / math.sqrt(64)
+        self.qp = O.pool_blocks(self.q)
+        self.kp = O.pool_blocks(self.k)
+        self.vp = O.pool_blocks(self.v)
+        self.P, self.vbar = O.block_scores(self.qp, self.kp, self.vp, self.scale)
+        self.gram = O.head_gram(O.to_numpy_f32(wl.w_o), self.H)
+        self.nb = self.P.shape[-1]
+        self.keep_k = wl.keep_k.cpu().numpy()
+        self.dense_q = wl.dense_q.cpu().numpy()
+        self.wl = wl
+
+    def drift_rows(self, rows):
+        s = {}
+        for (b, h, i) in rows:
+            s[(b, h, i)] = O.drift_row(self.P[b, h, i], self.vbar[b, h, i], self.vp[b, h], self.gram[h])
+        return s
+
+    def select(self, rows, method, rounds, seed, P=None, s_rows=None, vp=None, vbar=None):
+        P = self.P if P is None else P
+        vp = self.vp if vp is None else vp
+        vbar = self.vbar if vbar is None else vbar
+        s_full = None
+        if method == O.DRIFT:
+            s_full = np.zeros_like(P)
+            s_rows = s_rows if s_rows is not None else self.drift_rows(rows)
+            for r, val in s_rows.items():
+                s_full[r] = val
+        return O.select_blocks(method, P, self.wl.budgets, self.keep_k, self.dense_q, s=s_full,
+                               v_pool=vp, vbar=vbar, gram=self.gram, rounds=rounds,
+                               rho=self.wl.rho, eps=self.wl.eps, seed=seed, rows=rows)
+
+    def attention(self, kept, rows):
+        return O.block_sparse_attn(self.q, self.k, self.v, kept, self.scale, rows=rows)
+
+
+def close(got, want, rtol, atol, what):
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    err = np.abs(got - want)
+    lim = rtol * np.abs(want) + atol
+    bad = err > lim
+    assert not bad.any(), (f"{what}: {int(bad.sum())} of {bad.size} outside tolerance; "
+                           f"worst excess {float((err - lim).max()):.3g}")
+
+
+def check_drift(s_gpu_rows, orc: OracleLayer, rows):
+    s_orc = orc.drift_rows(rows)
+    for (b, h, i) in rows:
+        vb = orc.vbar[b, h, i].astype(np.float64)
+        M = orc.gram[h].astype(np.float64)
+        V = orc.vp[b, h].astype(np.float64)
+        a = vb @ M @ vb
+        bb = np.abs(V @ (M @ vb))
+        c = np.einsum("jd,de,je->j", V, M, V)
+        tol = orc.P[b, h, i] * np.sqrt(1e-6 * (a + 2 * bb + c))
+        close(s_gpu_rows[(b, h, i)], s_orc[(b, h, i)], 1e-4, tol + 1e-12, f"s{(b, h, i)}")
+
+
+def compare_masks(gpu_kept, orc_sel, nb, what):
+    """Kept lists identical on non-ambiguous rows; >= 99.9 % of mask bits agree."""
+    rows = sorted(orc_sel["kept"])
+    diff_bits, amb, mism = 0, 0, []
+    for r in rows:
+        g = set(gpu_kept[r])
+        o = set(orc_sel["kept"][r])
+        d = len(g ^ o)
+        diff_bits += d
+        if orc_sel["margin"][r] <= MARGIN:
+            amb += 1
+        elif d:
+            mism.append((r, sorted(g - o), sorted(o - g), orc_sel["margin"][r]))
+    agree = 1.0 - diff_bits / (len(rows) * nb)
+    assert not mism, f"{what}: {len(mism)} non-ambiguous rows differ, e.g. {mism[:3]}"
+    assert agree >= 0.999, f"{what}: mask agreement {agree:.5f}"
+    return dict(rows=len(rows), ambiguous=amb, agreement=agree)
+
+
+def check_attention(layer, orc: OracleLayer, rows):
+    kept = layer.kept_lists()
+    ref = orc.attention(kept, rows)
+    out = layer.out.float().cpu().numpy()
+    lse = layer.lse.cpu().numpy()
+    num, den, worst = 0.0, 0.0, 0.0
+    for (b, h, i) in rows:
+        o_ref, l_ref = ref[(b, h, i)]
+        r0 = i * 128
+        o_gpu = out[b, h, r0:r0 + o_ref.shape[0]]
+        worst = max(worst, float(np.abs(o_gpu - o_ref).max()))
+        num += float(((o_gpu - o_ref) ** 2).sum())
+        den += float((o_ref ** 2).sum())
+        l_gpu = lse[b, h, r0:r0 + o_ref.shape[0]]
+        if len(kept[(b, h, i)]):
+            close(l_gpu, l_ref, 1e-4, 1e-3, f"lse{(b, h, i)}")
+    rel = math.sqrt(num / max(den, 1e-30))
+    assert worst <= 2e-2, f"attention max-abs {worst:.4g}"
+    assert rel <= 1e-2, f"attention rel-L2 {rel:.4g}"
+    return worst, rel
+
+
+def sample_rows(B, H, nb, count, seed, always=()):
+    rng = np.random.default_rng(seed)
+    rows = set(always)
+    while len(rows) < min(count, B * H * nb):
+        rows.add((int(rng.integers(B)), int(rng.integers(H)), int(rng.integers(nb))))
+    return sorted(rows)

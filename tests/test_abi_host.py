@@ -1,0 +1,108 @@
+"""The C ABI on the host (no GPU): libress.so loads, exports every function that
+include/ress.h declares, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from block_sparse_global_b200 import build as B
+from block_sparse_global_b200 import ress as R
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "ress.h")
+INVALID, UNSUPPORTED, OK = 1, 2, 0
+FAKE = 0x7F0000000000  # 16-byte aligned, never dereferenced: every call below fails validation first
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return R.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ress_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_path(lib):
+    names = declared_functions()
+    for needed in ("ress_pool_blocks", "ress_block_scores", "ress_drift_scores",
+                   "ress_select_blocks", "ress_block_sparse_attn"):
+        assert needed in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"libress.so does not export {name}"
+
+
+def test_version_and_status_strings(lib):
+    assert R.ress_abi_version() == 1
+    assert R.ress_status_string(0) == "RESS_OK"
+    assert R.ress_status_string(5) == "RESS_ERR_DEVICE_TIMEOUT"
+    assert R.ress_status_string(99) == "RESS_ERR_UNKNOWN"
+
+
+def _pool(lib, shape, ptrs):
+    return lib.ress_pool_blocks(shape, *ptrs, None)
+
+
+def test_shape_validation(lib):
+    ptrs = [FAKE] * 6
+    assert _pool(lib, None, ptrs) == INVALID
+    assert _pool(lib, ctypes.byref(R.make_shape(1, 4, 1024, head_dim=128)), ptrs) == UNSUPPORTED
+    assert _pool(lib, ctypes.byref(R.make_shape(1, 4, 1024, block=64)), ptrs) == UNSUPPORTED
+    assert _pool(lib, ctypes.byref(R.make_shape(1, 129, 1024)), ptrs) == UNSUPPORTED
+    assert _pool(lib, ctypes.byref(R.make_shape(1, 4, 4096 * 128 + 1)), ptrs) == UNSUPPORTED
+    assert _pool(lib, ctypes.byref(R.make_shape(-1, 4, 1024)), ptrs) == INVALID
+    assert _pool(lib, ctypes.byref(R.make_shape(1, 0, 1024)), ptrs) == INVALID
+
+
+def test_empty_problem_is_ok_without_launch(lib):
+    for shape in (R.make_shape(0, 4, 1024), R.make_shape(2, 4, 0)):
+        assert _pool(lib, ctypes.byref(shape), [None] * 6) == OK
+        assert lib.ress_block_sparse_attn(ctypes.byref(shape), *([None] * 6), 0.125, None, None,
+                                          None, None) == OK
+
+
+def test_pointer_validation(lib):
+    shape = ctypes.byref(R.make_shape(1, 4, 1024))
+    assert _pool(lib, shape, [FAKE, FAKE, None, FAKE, FAKE, FAKE]) == INVALID
+    assert _pool(lib, shape, [FAKE + 8, FAKE, FAKE, FAKE, FAKE, FAKE]) == INVALID  # misaligned
+    assert lib.ress_block_scores(shape, FAKE, FAKE, FAKE, 0.0, FAKE, FAKE, None) == INVALID
+    assert lib.ress_block_scores(shape, FAKE, FAKE, FAKE, float("nan"), FAKE, FAKE, None) == INVALID
+    ws = lib.ress_drift_workspace_bytes(shape)
+    assert ws >= 4 * 8 * 66
+    assert lib.ress_drift_scores(shape, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ws - 1, None) == INVALID
+    assert lib.ress_attn_schedule(shape, FAKE, None, None) == INVALID
+    assert lib.ress_block_sparse_attn(shape, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 4, 0.125, FAKE,
+                                      None, None, None) == INVALID
+    assert lib.ress_head_gram(shape, 0, FAKE, FAKE, None) == INVALID
+
+
+def test_select_parameter_validation(lib):
+    shape = ctypes.byref(R.make_shape(1, 2, 1024))   # nb = 8
+    args = [FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None]
+
+    def call(method, budgets, rounds=2, rho=0.5, eps=1e-4):
+        p, keep = R.select_params(method, budgets, rounds=rounds, rho=rho, eps=eps)
+        return lib.ress_select_blocks(shape, ctypes.byref(p), *args)
+
+    assert call(1, [4, 9]) == INVALID             # budget > nb
+    assert call(1, [4, -1]) == INVALID
+    assert call(7, [4, 4]) == INVALID             # unknown method
+    assert call(1, [4, 4], rounds=65) == INVALID
+    assert call(1, [4, 4], rho=0.0) == INVALID
+    assert call(1, [4, 4], eps=0.0) == INVALID
+    p, keep = R.select_params(1, [4, 4], rounds=2)
+    assert lib.ress_select_blocks(shape, ctypes.byref(p), FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                  None, None, None) == INVALID          # drift needs s
+    assert lib.ress_select_blocks(shape, None, *args) == INVALID
+
+
+def test_python_binding_raises(lib):
+    with pytest.raises(R.RessError) as e:
+        R.ress_attn_schedule(R.make_shape(1, 4, 1024, head_dim=32), None, None)
+    assert e.value.status == UNSUPPORTED

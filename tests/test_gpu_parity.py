@@ -1,0 +1,232 @@
+"""CUDA path (through the C ABI) against the CPU oracle on the same seeded inputs.
+
+Small cases compare every element; the full-size VGGT-shaped layers compare the pooled
+tensors and P everywhere and drift, selection and attention on seeded row samples (plus
+the dense special-token rows).  Tolerances are documented in tests/parity.py."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_global_b200 import ress as R
+from block_sparse_global_b200 import workload as W
+from block_sparse_global_b200.pipeline import SparseGlobalAttention
+from oracle import ress_oracle as O
+from parity import (OracleLayer, check_attention, check_drift, close, compare_masks, ensure_built,
+                    run_gpu, sample_rows)
+
+pytestmark = pytest.mark.gpu
+METHODS = {"mass": O.MASS, "drift": O.DRIFT, "random": O.RANDOM}
+
+
+def _all_rows(B, H, nb):
+    return [(b, h, i) for b in range(B) for h in range(H) for i in range(nb)]
+
+
+def _check_block_tensors(layer, orc, rows_for_s=None):
+    close(layer.q_pool.cpu(), orc.qp, 1e-4, 1e-6, "q_pool")
+    close(layer.k_pool.cpu(), orc.kp, 1e-4, 1e-6, "k_pool")
+    close(layer.v_pool.cpu(), orc.vp, 1e-4, 1e-6, "v_pool")
+    close(layer.P.cpu(), orc.P, 1e-4, 1e-7, "P")
+    close(layer.v_bar.cpu(), orc.vbar, 1e-4, 1e-6, "v_bar")
+    close(layer.gram.cpu(), orc.gram, 1e-4, 1e-6, "gram")
+
+
+def _full_check(wl, method, rows, attn_rows, rounds=None):
+    layer = run_gpu(wl, method=method, rounds=rounds)
+    orc = OracleLayer(wl)
+    _check_block_tensors(layer, orc)
+    r = wl.rounds if rounds is None else rounds
+    if method != O.DRIFT:
+        r = 0
+    s_rows = None
+    if method == O.DRIFT:
+        s_gpu = layer.s.cpu().numpy()
+        check_drift({row: s_gpu[row] for row in rows}, orc, rows)
+        s_rows = orc.drift_rows(rows)
+    sel = orc.select(rows, method, r, wl.select_seed, s_rows=s_rows)
+    kept = layer.kept_lists()
+    stats = compare_masks(kept, sel, orc.nb, f"{wl.case.name}/{method}")
+    mask = layer.mask.cpu().numpy()
+    for (b, h, i) in rows:
+        assert sorted(np.nonzero(mask[b, h, i])[0].tolist()) == kept[(b, h, i)]
+    check_attention(layer, orc, attn_rows)
+    return layer, orc, stats
+
+
+@pytest.mark.parametrize("method", ["mass", "drift", "random"])
+def test_tiny_case_every_element(method):
+    wl = W.make_workload(1)
+    rows = _all_rows(1, 4, 8)
+    layer, orc, stats = _full_check(wl, METHODS[method], rows, rows)
+    assert all(len(v) == 4 for v in layer.kept_lists().values())
+
+
+@pytest.mark.parametrize("method", ["mass", "drift", "random"])
+def test_small_vggt_layer_with_specials_and_ragged_tail(method):
+    # 3 views: N = 4122, 33 blocks, last block 26 tokens, 15 special tokens -> block 32
+    wl = W.make_workload(2, heads=2, views=3, method=method, sparsity=0.6, rounds=4)
+    rows = _all_rows(1, 2, wl.nb)
+    layer, orc, stats = _full_check(wl, METHODS[method], rows, rows, rounds=4)
+    kept = layer.kept_lists()
+    for (b, h, i), k in kept.items():
+        assert (wl.nb - 1) in k
+        if i == wl.nb - 1:
+            assert k == list(range(wl.nb))
+
+
+def test_selection_alone_on_oracle_scores():
+    """Feed the oracle's own P, s, pooled values and Gram to the GPU selection: this
+    isolates the selection arithmetic (top-k, Eqs. 13-17, track-best)."""
+    wl = W.make_workload(2, heads=4, views=6, method="drift", sparsity=0.75, rounds=5)
+    ensure_built()
+    orc = OracleLayer(wl)
+    rows = _all_rows(1, 4, orc.nb)
+    s_rows = orc.drift_rows(rows)
+    s = np.zeros_like(orc.P)
+    for r, val in s_rows.items():
+        s[r] = val
+    dev = torch.device("cuda")
+    layer = SparseGlobalAttention(1, 4, wl.q.shape[2], device=dev, with_mask=True)
+    layer.P.copy_(torch.from_numpy(orc.P))
+    layer.s.copy_(torch.from_numpy(s))
+    layer.v_pool.copy_(torch.from_numpy(orc.vp))
+    layer.v_bar.copy_(torch.from_numpy(orc.vbar))
+    layer.gram.copy_(torch.from_numpy(orc.gram))
+    for method, rounds in ((O.MASS, 0), (O.DRIFT, 0), (O.DRIFT, 5), (O.RANDOM, 0)):
+        layer.select(method, wl.budgets, wl.keep_k.to(dev), wl.dense_q.to(dev), rounds, wl.rho,
+                     wl.eps, wl.select_seed)
+        torch.cuda.synchronize()
+        sel = orc.select(rows, method, rounds, wl.select_seed, s_rows=s_rows)
+        stats = compare_masks(layer.kept_lists(), sel, orc.nb, f"selection-only/{method}/{rounds}")
+        if method == O.RANDOM:
+            assert stats["agreement"] == 1.0
+
+
+def test_vggt_8view_mass50_full_layer():
+    wl = W.make_workload(2)
+    nb = wl.nb
+    rows = _all_rows(1, 16, nb)
+    attn_rows = sample_rows(1, 16, nb, 40, seed=1, always=[(0, h, nb - 1) for h in (0, 15)])
+    layer, orc, stats = _full_check(wl, O.MASS, rows, attn_rows)
+    cnt = layer.kv_cnt.cpu()
+    assert int(cnt[0, 0, 0]) == 43 + 1 and int(cnt[0, 3, nb - 1]) == nb
+
+
+def test_vggt_32view_drift75_r3():
+    wl = W.make_workload(3)
+    nb = wl.nb
+    rows = sample_rows(1, 16, nb, 64, seed=2, always=[(0, 0, nb - 1), (0, 7, 0)])
+    attn_rows = sample_rows(1, 16, nb, 16, seed=3, always=[(0, 5, nb - 2)])
+    _full_check(wl, O.DRIFT, rows, attn_rows)
+
+
+def test_vggt_100view_drift90_r5_dirichlet():
+    wl = W.make_workload(4)
+    nb = wl.nb
+    assert sum(wl.budgets) == 16 * 107
+    rows = sample_rows(1, 16, nb, 48, seed=4, always=[(0, 2, nb - 1)])
+    attn_rows = sample_rows(1, 16, nb, 12, seed=5, always=[(0, 9, nb - 3)])
+    layer, orc, stats = _full_check(wl, O.DRIFT, rows, attn_rows)
+    cnt = layer.kv_cnt.cpu()
+    for h in range(16):
+        assert int(cnt[0, h, 0]) == min(wl.budgets[h], nb - 5) + 5
+
+
+@pytest.mark.parametrize("layer_id,sparsity,method", [(0, 0.0, "mass"), (0, 0.9, "random"),
+                                                       (23, 0.25, "drift"), (11, 0.5, "mass")])
+def test_vggt_64view_sweep_points(layer_id, sparsity, method):
+    wl = W.make_workload(5, layer=layer_id, method=method, sparsity=sparsity)
+    nb = wl.nb
+    rows = sample_rows(1, 16, nb, 24, seed=layer_id + 10)
+    attn_rows = sample_rows(1, 16, nb, 8, seed=layer_id + 20)
+    _full_check(wl, METHODS[method], rows, attn_rows)
+
+
+def test_keep_all_is_dense_attention():
+    """Sparsity 0 keeps every block: the kernel computes dense attention; compare with
+    torch SDPA in fp32 on a sample of query blocks (library routine, same definition)."""
+    wl = W.make_workload(2, heads=4, views=4, method="mass", sparsity=0.0)
+    layer = run_gpu(wl)
+    assert int(layer.kv_cnt.min()) == wl.nb
+    q, k, v = (t.cuda().float() for t in (wl.q, wl.k, wl.v))
+    ref = torch.nn.functional.scaled_dot_product_attention(q, k, v, scale=0.125)
+    err = (layer.out.float() - ref).abs().max().item()
+    rel = ((layer.out.float() - ref).norm() / ref.norm()).item()
+    assert err <= 2e-2 and rel <= 1e-2, (err, rel)
+
+
+def _manual_attn(N, lists, B=1, H=2, seed=0):
+    ensure_built()
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    q, k, v = (torch.randn(B, H, N, 64, device="cuda", generator=g).to(torch.bfloat16)
+               for _ in range(3))
+    nb = (N + 127) // 128
+    kv_idx = torch.zeros(B, H, nb, nb, dtype=torch.int32)
+    kv_cnt = torch.zeros(B, H, nb, dtype=torch.int32)
+    for (b, h, i), lst in lists.items():
+        kv_cnt[b, h, i] = len(lst)
+        kv_idx[b, h, i, :len(lst)] = torch.tensor(lst, dtype=torch.int32)
+    out = torch.full((B, H, N, 64), 7.0, device="cuda", dtype=torch.bfloat16)
+    lse = torch.empty(B, H, N, device="cuda")
+    err = torch.zeros(1, device="cuda", dtype=torch.int32)
+    R.ress_block_sparse_attn(R.make_shape(B, H, N), q, k, v, kv_idx.cuda(), kv_cnt.cuda(), None,
+                             0.125, out, lse, err)
+    torch.cuda.synchronize()
+    return q, k, v, out, lse, int(err.item())
+
+
+def test_edge_rows_empty_unsorted_single_partial_block():
+    N = 300   # 3 blocks, last one 44 tokens
+    lists = {(0, 0, 0): [2, 0], (0, 0, 1): [], (0, 0, 2): [2], (0, 1, 0): [0, 1, 2],
+             (0, 1, 1): [1], (0, 1, 2): [1, 2, 0]}
+    q, k, v, out, lse, err = _manual_attn(N, lists)
+    assert err == 0
+    qn, kn, vn = (O.to_numpy_f32(t) for t in (q, k, v))
+    for (b, h, i), lst in lists.items():
+        o_ref, l_ref = O.attention_qblock(qn, kn, vn, b, h, i, sorted(lst), 0.125)
+        o = out[b, h, i * 128:i * 128 + o_ref.shape[0]].float().cpu().numpy()
+        assert np.abs(o - o_ref).max() <= 2e-2
+        if not lst:
+            assert np.all(o == 0) and torch.isinf(lse[b, h, 128:256]).all()
+
+
+def test_tiny_sequence_below_one_block():
+    lists = {(b, h, 0): [0] for b in range(2) for h in range(2)}
+    q, k, v, out, lse, err = _manual_attn(100, lists, B=2)
+    ref = torch.nn.functional.scaled_dot_product_attention(q.float(), k.float(), v.float(), scale=0.125)
+    assert err == 0 and (out.float() - ref).abs().max().item() <= 2e-2
+
+
+def test_out_of_range_kv_index_sets_device_error_and_skips_row():
+    lists = {(0, 0, 0): [0, 5], (0, 0, 1): [1], (0, 1, 0): [0], (0, 1, 1): [0, 1]}
+    q, k, v, out, lse, err = _manual_attn(256, lists)
+    assert err == 4   # RESS_ERR_DEVICE_BOUNDS
+    assert torch.all(out[0, 0, :128].float() == 7.0)       # the bad row is left unwritten
+    assert not torch.all(out[0, 1, :128].float() == 7.0)   # the others are computed
+
+
+def test_repeat_runs_are_bit_identical():
+    """Two runs on the same inputs give the same bytes (ReSS Supp. B.4 reports the same)."""
+    wl = W.make_workload(3, heads=4, views=5, method="drift", rounds=5)
+    a = run_gpu(wl)
+    b = run_gpu(wl)
+    for name in ("q_pool", "P", "v_bar", "s", "kv_cnt", "mask", "out", "lse"):
+        assert torch.equal(getattr(a, name), getattr(b, name)), name
+    for bb, h, i in _all_rows(1, 4, wl.nb):
+        c = int(a.kv_cnt[bb, h, i])
+        assert torch.equal(a.kv_idx[bb, h, i, :c], b.kv_idx[bb, h, i, :c])
+
+
+def test_schedule_is_a_stable_descending_permutation():
+    ensure_built()
+    g = torch.Generator().manual_seed(0)
+    shape = R.make_shape(2, 3, 1000)   # nb = 8, 48 items
+    cnt = torch.randint(0, 9, (2, 3, 8), generator=g, dtype=torch.int32)
+    order = torch.empty(48, dtype=torch.int32, device="cuda")
+    R.ress_attn_schedule(shape, cnt.cuda(), order)
+    torch.cuda.synchronize()
+    flat = cnt.flatten().tolist()
+    want = sorted(range(48), key=lambda it: (-flat[it], it))
+    assert order.cpu().tolist() == want
