@@ -1,0 +1,425 @@
+#!/usr/bin/env python
+"""Benchmark of one block-sparse global-attention layer on B200 (one JSON line).
+
+A step is one pass of the whole path over one layer of synthetic VGGT-shaped input:
+pool -> pooled block map -> (drift) -> selection -> schedule -> block-sparse attention.
+Default workload: 8 views x 1374 tokens (10992), 16 heads, head_dim 64, block 128, 50 %
+sparsity, attention-mass selection.  `--case 3/4` runs the drift workloads instead.
+
+    python bench.py [--gpus N --steps K --warmup W] [--case 2] [--impl reference]
+
+value      whole-job effective TFLOP/s over kept tiles (kept-tile FLOPs of all ranks /
+           max over ranks of the summed per-step device time); inputs resident in HBM,
+           L2 flushed (256 MiB write) before every timed step.
+e2e        the same metric with Q, K, V copied from pinned host memory and the output
+           copied back inside every timed step.
+roofline   the attention kernel (dominant): kept-tile FLOPs per launch / its mean CUDA-
+           event duration, against the measured dense bf16 tensor-core peak.
+With N > 1 (torchrun) every rank runs its own layer (independent seeds): weak scaling,
+no collective on the data path.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "global-attn layer latency (ms) & effective TFLOP/s on kept tiles vs bf16 peak"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_BF16_TFLOPS = 1590.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--case", type=int, default=2, help="synthetic case index (2 = 8 views, mass 50%%)")
+    ap.add_argument("--method", choices=["mass", "drift", "random"], default=None)
+    ap.add_argument("--sparsity", type=float, default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--quick", action="store_true", help="timed loop only (profiling runs)")
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops"]), float(p.get("hbm_gbs", 0.0)), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        mhz = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        maxmhz = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k].lower() == "active"})
+        loaded = [m for m in mhz if m > 0.5 * max(mhz)] if mhz else []
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(maxmhz) if maxmhz else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------- workload
+def build_case(args, rank: int):
+    from block_sparse_global_b200 import workload as W
+    return W.make_workload(args.case, layer=rank, device="cuda", method=args.method,
+                           sparsity=args.sparsity)
+
+
+def kept_tile_flops(kv_idx, kv_cnt, N: int) -> float:
+    """Algorithmic FLOPs over kept tiles: sum of 4 * rows * cols * 64 (QK^T and PV), rows
+    and cols counting only tokens < N."""
+    import torch
+    B, H, nb, _ = kv_idx.shape
+    ar = torch.arange(nb, device=kv_idx.device)
+    valid = torch.clamp(N - ar * 128, max=128).to(torch.float64)          # tokens per block
+    pos = torch.arange(nb, device=kv_idx.device).view(1, 1, 1, nb)
+    live = pos < kv_cnt.unsqueeze(-1)
+    cols = torch.where(live, valid[kv_idx.clamp(0, nb - 1).long()], torch.zeros((), dtype=torch.float64,
+                                                                             device=kv_idx.device))
+    per_row = cols.sum(-1) * valid.view(1, 1, nb)
+    return float(per_row.sum().item()) * 4.0 * 64.0
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from block_sparse_global_b200 import build as B
+    from block_sparse_global_b200 import ress as R
+    from block_sparse_global_b200.pipeline import SparseGlobalAttention
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if rank == 0:
+        B.build()
+    if world > 1:
+        dist.barrier()
+    R.load()
+
+    wl = build_case(args, rank)
+    Bsz, H, N, _ = wl.q.shape
+    q, k, v = wl.q, wl.k, wl.v
+    keep_k, dense_q = wl.keep_k, wl.dense_q
+    layer = SparseGlobalAttention(Bsz, H, N, device=dev)
+    layer.load_output_projection(wl.w_o)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, device=dev, dtype=torch.float32)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        layer.scores(q, k, v)
+        if wl.method == R.SELECT_DRIFT:
+            layer.drift()
+        layer.select(wl.method, wl.budgets, keep_k, dense_q, wl.rounds, wl.rho, wl.eps, wl.select_seed)
+        R.ress_attn_schedule(layer.shape, layer.kv_cnt, layer.order)
+
+    def attn():
+        R.ress_block_sparse_attn(layer.shape, q, k, v, layer.kv_idx, layer.kv_cnt, layer.order,
+                                 layer.scale, layer.out, layer.lse, layer.dev_err)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step()
+        attn()
+    torch.cuda.synchronize()
+    if layer.device_error():
+        raise SystemExit(f"device error {layer.device_error()} during warm-up")
+    flops = kept_tile_flops(layer.kv_idx, layer.kv_cnt, N)
+    kept_frac = float(layer.kv_cnt.sum().item()) / (Bsz * H * layer.nb * layer.nb)
+
+    clocks = ClockSampler(local)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    for s in range(args.steps):
+        flush.fill_(1.0)
+        ev[s][0].record(stream)
+        step()
+        ev[s][1].record(stream)
+        attn()
+        ev[s][2].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    step_ms = [e[0].elapsed_time(e[2]) for e in ev]
+    attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    total_ms = sum(step_ms)
+    t = torch.tensor([total_ms, flops * args.steps], dtype=torch.float64, device=dev)
+    if world > 1:
+        tmax = t[:1].clone()
+        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
+        fsum = t[1:].clone()
+        dist.all_reduce(fsum, op=dist.ReduceOp.SUM)
+        total_ms_max, flops_all = float(tmax.item()), float(fsum.item())
+    else:
+        total_ms_max, flops_all = total_ms, flops * args.steps
+    value = flops_all / (total_ms_max * 1e-3) / 1e12
+
+    extra = {}
+    if not args.quick:
+        # per-kernel breakdown (separate pass, same inputs)
+        names = ["pool", "block_scores", "drift", "select", "schedule", "attention"]
+        calls = {
+            "pool": lambda: R.ress_pool_blocks(layer.shape, q, k, v, layer.q_pool, layer.k_pool, layer.v_pool),
+            "block_scores": lambda: R.ress_block_scores(layer.shape, layer.q_pool, layer.k_pool, layer.v_pool,
+                                                        layer.scale, layer.P, layer.v_bar),
+            "drift": layer.drift,
+            "select": lambda: layer.select(wl.method, wl.budgets, keep_k, dense_q, wl.rounds, wl.rho,
+                                           wl.eps, wl.select_seed),
+            "schedule": lambda: R.ress_attn_schedule(layer.shape, layer.kv_cnt, layer.order),
+            "attention": attn,
+        }
+        per = {}
+        for name in names:
+            if name == "drift" and wl.method != R.SELECT_DRIFT:
+                continue
+            times = []
+            for _ in range(5):
+                flush.fill_(1.0)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                calls[name]()
+                b.record(stream)
+                torch.cuda.synchronize()
+                times.append(a.elapsed_time(b))
+            per[name] = round(statistics.median(times), 4)
+        extra["kernels_ms"] = per
+        # same-shape dense attention: every query block keeps every key block
+        dense_idx = torch.arange(layer.nb, device=dev, dtype=torch.int32).expand(Bsz, H, layer.nb, layer.nb).contiguous()
+        dense_cnt = torch.full((Bsz, H, layer.nb), layer.nb, device=dev, dtype=torch.int32)
+        dense_out = torch.empty_like(layer.out)
+        dts = []
+        for _ in range(5):
+            flush.fill_(1.0)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            R.ress_block_sparse_attn(layer.shape, q, k, v, dense_idx, dense_cnt, None, layer.scale, dense_out)
+            b.record(stream)
+            torch.cuda.synchronize()
+            dts.append(a.elapsed_time(b))
+        dense_flops = kept_tile_flops(dense_idx, dense_cnt, N)
+        dms = statistics.median(dts)
+        extra["dense_attention"] = {"ms": round(dms, 4), "tflops": round(dense_flops / dms / 1e9, 1)}
+        del dense_idx, dense_cnt, dense_out
+        # end to end through the API with host buffers
+        if not args.no_e2e:
+            qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
+            outh = torch.empty(layer.out.shape, dtype=layer.out.dtype).pin_memory()
+            qd, kd, vd = (torch.empty_like(x) for x in (q, k, v))
+            e2e_ms = []
+            for s in range(max(3, args.steps // 2) + 2):
+                flush.fill_(1.0)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                qd.copy_(qh, non_blocking=True)
+                kd.copy_(kh, non_blocking=True)
+                vd.copy_(vh, non_blocking=True)
+                layer.forward(qd, kd, vd, wl.method, wl.budgets, keep_k, dense_q, wl.rounds, wl.rho,
+                              wl.eps, wl.select_seed)
+                outh.copy_(layer.out, non_blocking=True)
+                b.record(stream)
+                torch.cuda.synchronize()
+                if s >= 2:
+                    e2e_ms.append(a.elapsed_time(b))
+            em = statistics.mean(e2e_ms)
+            extra["e2e"] = {"value": round(flops / (em * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                            "ms_per_step": round(em, 4),
+                            "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
+                            "d2h_bytes_per_step": layer.out.numel() * layer.out.element_size()}
+    bf16_peak, hbm_peak, peak_kind = peaks()
+    attn_mean = statistics.mean(attn_ms)
+    achieved = flops / (attn_mean * 1e-3) / 1e12
+    line = {
+        "metric": METRIC,
+        "value": round(value, 3),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms_max / args.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded, VGGT-shaped)",
+        "config": {
+            "workload": wl.case.name, "batch": Bsz, "heads": H, "seq_len": N, "head_dim": 64,
+            "block": 128, "method": ["mass", "drift", "random"][wl.method], "sparsity": wl.sparsity,
+            "rounds": wl.rounds, "budgets": sorted(set(wl.budgets)) if len(set(wl.budgets)) < 4 else "dirichlet",
+            "kept_tile_fraction": round(kept_frac, 4), "kept_tile_gflop": round(flops / 1e9, 3),
+            "selection_dtype": "f32", "l2": "flushed before every timed step (256 MiB write)",
+            "parallelism": f"{world} independent layers, one per GPU" if world > 1 else "single GPU",
+        },
+        "roofline": {"kernel": "block_sparse_attn", "bound": "tensor", "achieved": round(achieved, 2),
+                     "peak": bf16_peak, "unit": "TFLOP/s", "frac": round(achieved / bf16_peak, 4),
+                     "peak_source": f"{peak_kind} dense bf16 (burst)", "traffic": None,
+                     "mean_launch_ms": round(attn_mean, 4)},
+        "gpu_launches": args.steps * layer.kernel_launches(wl.method),
+    }
+    if clk:
+        line["clocks"] = clk
+    line.update({k_: v_ for k_, v_ in extra.items() if k_ != "e2e"})
+    if "e2e" in extra:
+        line["e2e"] = extra["e2e"]
+    if rank == 0 and not args.no_cpu_baseline and world == 1 and not args.quick:
+        line["cpu_baseline"] = cpu_baseline(wl, seconds=15.0)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------- CPU oracle timing
+def _oracle_sample(wl, heads):
+    """Runs the oracle's whole path for the listed heads of the layer; returns
+    (seconds, kept-tile FLOPs of the sample)."""
+    import numpy as np
+
+    from oracle import ress_oracle as O
+    q = O.to_numpy_f32(wl.q)[:, heads]
+    k = O.to_numpy_f32(wl.k)[:, heads]
+    v = O.to_numpy_f32(wl.v)[:, heads]
+    w_cols = np.concatenate([np.arange(64 * h, 64 * h + 64) for h in heads])
+    w_o = O.to_numpy_f32(wl.w_o)[:, w_cols]
+    budgets = [wl.budgets[h] for h in heads]
+    t0 = time.perf_counter()
+    res = O.layer(q, k, v, w_o, wl.method, budgets, wl.keep_k.cpu().numpy(), wl.dense_q.cpu().numpy(),
+                  rounds=wl.rounds, rho=wl.rho, eps=wl.eps, seed=wl.select_seed)
+    dt = time.perf_counter() - t0
+    N = q.shape[2]
+    valid = [min(128, N - 128 * j) for j in range((N + 127) // 128)]
+    fl = sum(4.0 * 64 * valid[i] * sum(valid[j] for j in kept) for (b, h, i), kept in res["kept"].items())
+    return dt, fl
+
+
+def _cores():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((int(x.get("num_threads", 1)) for x in threadpool_info()), default=1)
+        return max(1, n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(wl, seconds: float = 15.0):
+    H = wl.q.shape[1]
+    done, tot_t, tot_f, h = [], 0.0, 0.0, 0
+    while tot_t < seconds and h < H:
+        dt, fl = _oracle_sample(wl, [h])
+        tot_t += dt
+        tot_f += fl
+        done.append(h)
+        h += 1
+    return {"value": round(tot_f / tot_t / 1e12, 6), "unit": "TFLOP/s", "cores": _cores(),
+            "kind": "oracle",
+            "sample": f"whole path (pool, block map, {'drift, ' if wl.method == 1 else ''}selection, "
+                      f"attention) for {len(done)} of {H} heads of the same layer, "
+                      f"{tot_t:.1f} s of host time"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    import torch
+    from block_sparse_global_b200 import workload as W
+    wl = W.make_workload(args.case, layer=0, device="cpu", method=args.method, sparsity=args.sparsity)
+    H = wl.q.shape[1]
+    times, flops = [], []
+    for s in range(args.warmup + args.steps):
+        dt, fl = _oracle_sample(wl, [s % H])
+        if s >= args.warmup:
+            times.append(dt)
+            flops.append(fl)
+    value = sum(flops) / sum(times) / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * statistics.mean(times), 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded, VGGT-shaped)",
+        "config": {"workload": wl.case.name, "batch": 1, "heads": H, "seq_len": wl.q.shape[2],
+                   "head_dim": 64, "block": 128, "method": ["mass", "drift", "random"][wl.method],
+                   "sparsity": wl.sparsity, "rounds": wl.rounds,
+                   "step": "oracle whole path for one head of the layer (heads rotate)"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
+                         "sample": "one of the layer's heads per step, whole path"},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()
