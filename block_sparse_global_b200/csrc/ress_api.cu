@@ -209,3 +209,55 @@ ress_status ress_block_sparse_attn(const ress_shape *shape, const void *q, const
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------------
+// ress_drift_scores_static: the drift score for callers that cannot allocate device
+// memory.  Its scratch is this file's static device array; the host looks up the array's
+// device address once per device (the array's name in host code is only a stand-in).
+#include <mutex>
+
+namespace {
+
+constexpr size_t kDriftStaticBytes = (size_t)8 << 20;  // 8 MiB, see include/ress.h
+static __device__ __align__(256) unsigned char g_drift_static_scratch[kDriftStaticBytes];
+
+constexpr int kMaxDevices = 64;
+void *g_drift_static_addr[kMaxDevices] = {};
+std::mutex g_drift_static_mu;
+
+// Device address of the static scratch on the current device; looked up on the first
+// call per device, with that device current.
+cudaError_t drift_static_address(void **out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_drift_static_mu);
+  if (g_drift_static_addr[dev] == nullptr) {
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_drift_static_scratch);
+    if (e != cudaSuccess) return e;
+    g_drift_static_addr[dev] = p;
+  }
+  *out = g_drift_static_addr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" ress_status ress_drift_scores_static(const ress_shape *shape, const float *P,
+                                                const float *v_pool, const float *v_bar,
+                                                const float *gram, float *s,
+                                                ress_stream_t stream) {
+  Dims d;
+  bool empty;
+  ress_status st = check_shape(shape, &d, &empty);
+  if (st != RESS_OK) return st;
+  if (empty) return RESS_OK;
+  if (!ptr_ok(P) || !ptr_ok(v_pool) || !ptr_ok(v_bar) || !ptr_ok(gram) || !ptr_ok(s))
+    return RESS_ERR_INVALID_ARG;
+  if (ress::drift_workspace_bytes(d) > kDriftStaticBytes) return RESS_ERR_UNSUPPORTED;
+  void *scratch = nullptr;
+  if (drift_static_address(&scratch) != cudaSuccess) return RESS_ERR_CUDA;
+  return from_cuda(ress::launch_drift(d, P, v_pool, v_bar, gram, s, scratch, (cudaStream_t)stream));
+}

@@ -55,6 +55,7 @@ _SIGS = {
     "ress_drift_workspace_bytes": (_SZ, [ctypes.POINTER(ress_shape)]),
     "ress_drift_scores": (_I32, [ctypes.POINTER(ress_shape), _VP, _VP, _VP, _VP, _VP, _VP, _SZ,
                                  _VP]),
+    "ress_drift_scores_static": (_I32, [ctypes.POINTER(ress_shape), _VP, _VP, _VP, _VP, _VP, _VP]),
     "ress_select_blocks": (_I32, [ctypes.POINTER(ress_shape), ctypes.POINTER(ress_select_params),
                                   _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     "ress_attn_schedule": (_I32, [ctypes.POINTER(ress_shape), _VP, _VP, _VP]),
@@ -149,6 +150,14 @@ def ress_drift_scores(shape, P, v_pool, v_bar, gram, s, workspace: torch.Tensor,
     st = load().ress_drift_scores(ctypes.byref(_shape(shape)), _ptr(P), _ptr(v_pool), _ptr(v_bar),
                                   _ptr(gram), _ptr(s), _ptr(workspace), nbytes, _stream(stream))
     _check("ress_drift_scores", st)
+
+
+def ress_drift_scores_static(shape, P, v_pool, v_bar, gram, s, stream=None):
+    """Drift score with the library's fixed static scratch (no workspace argument), for
+    callers that cannot allocate device memory; see include/ress.h."""
+    st = load().ress_drift_scores_static(ctypes.byref(_shape(shape)), _ptr(P), _ptr(v_pool),
+                                         _ptr(v_bar), _ptr(gram), _ptr(s), _stream(stream))
+    _check("ress_drift_scores_static", st)
 
 
 def select_params(method: int, budgets: Sequence[int], keep_k=None, dense_q=None, rounds: int = 0,

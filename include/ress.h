@@ -168,6 +168,33 @@ ress_status ress_drift_scores(const ress_shape *shape, const float *P, const flo
                               ress_stream_t stream);
 
 /*
+ * ress_drift_scores_static -- the drift score of ress_drift_scores for callers that cannot
+ * allocate device memory.  Some callers receive only their inputs and outputs: the
+ * plugin interface of an inference engine that offers no workspace, or a runtime that
+ * reserves all device memory at start-up and forbids cudaMalloc / cudaFree afterwards
+ * (those calls synchronise the device, and can fail or fragment memory in the middle of
+ * a run).  This call takes no workspace: its scratch is a fixed 8 MiB buffer inside
+ * libress.so, a static device array that every GPU which loads the library holds until
+ * the process exits.  The paper has no counterpart to this call; it exists only for
+ * such callers.
+ *   Arguments, layouts and results are those of ress_drift_scores, minus the workspace.
+ *   Limit: a shape whose ress_drift_workspace_bytes(shape) exceeds 8 MiB (8,388,608
+ *   bytes; about 31,700 pooled rows B*H*nb) is rejected with RESS_ERR_UNSUPPORTED before
+ *   anything is launched.
+ *   The first call on each device looks up the buffer's device address with a CUDA
+ *   runtime call, made with that device current; make this first call before any stream
+ *   capture.
+ *   Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ *   All calls on a device share the one buffer, which keeps the last call's contents
+ *   (each call writes every part of it that it later reads, so nothing needs clearing).
+ *   Calls that overlap on the GPU -- on different streams, or from threads whose calls
+ *   are not ordered -- race on the buffer and give wrong results: order them.
+ */
+ress_status ress_drift_scores_static(const ress_shape *shape, const float *P,
+                                     const float *v_pool, const float *v_bar,
+                                     const float *gram, float *s, ress_stream_t stream);
+
+/*
  * ress_select_blocks -- per (query block, head) key-block selection ([ReSS] §4.1 Eq. 2,
  * §4.2 Eq. 7, §4.3 Eqs. 10-17; SparseVGGT/HeSS attention-mass top-k).
  * Candidates are the key blocks with keep_k == 0.  A row whose dense_q flag is set
