@@ -9,14 +9,20 @@
 //   warps 0-3  softmax: thread t owns query row t (tensor-memory lane t).  Reads the
 //              S tile from tensor memory, online softmax in the exp2 domain, writes P
 //              (bf16) back to tensor memory, rescales O when the running max grows by
-//              more than 2^8, and runs the epilogue (O / l -> bf16, LSE).
-//   warp 4     TMA producer: Q once, then K_j and V_j of every kept block into a
-//              two-stage shared-memory ring.
+//              more than a factor 2^8, and runs the epilogue (O / l -> bf16, LSE).
+//   warp 4     TMA producer (one thread): Q once, then K_j of every kept block into a
+//              three-slot ring and V_j into a two-slot ring; validates the row first.
 //   warp 5     tensor-core issuer (one elected thread): S = Q K^T (M=128, N=128, K=64)
 //              and O += P V (M=128, N=64, K=128, A operand read from tensor memory).
 //              Also allocates and frees the 256 tensor-memory columns.
 // Tensor memory: S columns [0,128), P [128,192) as packed bf16 pairs, O [192,256).
-// Shared memory: Q 16 KB, K 2 x 16 KB, V 2 x 16 KB, all 128-byte swizzled by TMA.
+// Shared memory: Q 16 KB, K 3 x 16 KB, V 2 x 16 KB, all 128-byte swizzled by TMA.
+//
+// Exponentials: at head_dim 64 the MUFU unit (about 16-21 exp2 per clock per SM) is the
+// scarcest resource of the softmax -- a 128 x 128 tile needs 16384 exp2 against roughly
+// 700 clock cycles of tensor-core work.  Two of every eight column pairs therefore take
+// exp2 on the FMA and integer pipes instead (range reduction plus a fitted polynomial,
+// see exp2_pair_fma); the rest use MUFU ex2.approx.f32.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -30,20 +36,27 @@ namespace ress {
 namespace {
 
 constexpr int kThreads = 192;
-constexpr int kStages = 2;
+constexpr int kProducerWarp = 4;
+constexpr int kMmaWarp = 5;
+// lazy rescale: O and l are rescaled only when the row max grows by more than 2^this
+constexpr float kRescaleLog2 = 8.0f;
+constexpr int kKStages = 3;          // K tiles in flight (S = Q K^T consumes them first)
+constexpr int kVStages = 2;          // V tiles in flight (O += P V consumes them later)
 constexpr int kTile = 128 * 64 * 2;  // bytes of one 128 x 64 bf16 tile
 constexpr int kOffQ = 0;
 constexpr int kOffK = kTile;
-constexpr int kOffV = kOffK + kStages * kTile;
-constexpr int kOffBar = kOffV + kStages * kTile;
-constexpr int kSmemBytes = kOffBar + 256 + 1024;  // + barriers + alignment slack
+constexpr int kOffV = kOffK + kKStages * kTile;
+constexpr int kOffBar = kOffV + kVStages * kTile;
+constexpr int kSmemBytes = kOffBar + 256 + 1024;  // + barriers, alignment slack
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColS = 0, kColP = 128, kColO = 192;
 
 struct Bars {
   uint64_t q_full;
-  uint64_t kv_full[kStages];
-  uint64_t kv_empty[kStages];
+  uint64_t k_full[kKStages];
+  uint64_t k_empty[kKStages];
+  uint64_t v_full[kVStages];
+  uint64_t v_empty[kVStages];
   uint64_t s_full;
   uint64_t s_free;
   uint64_t p_full;
@@ -59,6 +72,59 @@ RESS_DEV uint64_t smem_desc(uint32_t saddr) {
   return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)64 << 32) |
          ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
+
+// ---------------------------------------------------------------- softmax arithmetic
+// Two fp32 values in one 64-bit register, for the packed f32x2 FMA-pipe instructions.
+RESS_DEV uint64_t f2(float lo, float hi) {
+  return ((uint64_t)__float_as_uint(hi) << 32) | __float_as_uint(lo);
+}
+RESS_DEV float f2lo(uint64_t v) { return __uint_as_float((uint32_t)v); }
+RESS_DEV float f2hi(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
+RESS_DEV uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+RESS_DEV uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+RESS_DEV float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for a pair, on the FMA / integer pipes instead of the MUFU unit.  Range reduction
+// to nearest: x = j + f with j = round(x) (adding 1.5 * 2^23 rounds to an integer in the
+// low mantissa bits), f in [-1/2, 1/2]; 2^f from a degree-3 polynomial fitted here for
+// minimax relative error over [-1/2, 1/2] (Lawson's iteratively reweighted least squares,
+// max relative error 7.5e-5, far below the bf16 rounding P receives); 2^j enters by
+// adding j to the exponent field.  x is clamped at -126 first (masked logits are -inf):
+// the polynomial value lies in [0.70, 1.42], so j >= -126 keeps the exponent field >= 0.
+constexpr float kPoly0 = 0.99992805719f, kPoly1 = 0.69326096773f, kPoly2 = 0.24261116982f,
+                kPoly3 = 0.05517166480f;
+constexpr float kRoundMagic = 12582912.0f;
+RESS_DEV uint64_t exp2_pair_fma(uint64_t x) {
+  const float lo = fmaxf(f2lo(x), -126.0f), hi = fmaxf(f2hi(x), -126.0f);
+  x = f2(lo, hi);
+  const uint64_t t = fadd2(x, f2(kRoundMagic, kRoundMagic));
+  const uint64_t r = fadd2(t, f2(-kRoundMagic, -kRoundMagic));
+  const uint64_t f = ffma2(r, f2(-1.0f, -1.0f), x);
+  uint64_t q = ffma2(f, f2(kPoly3, kPoly3), f2(kPoly2, kPoly2));
+  q = ffma2(q, f, f2(kPoly1, kPoly1));
+  q = ffma2(q, f, f2(kPoly0, kPoly0));
+  const uint32_t qlo = (uint32_t)q + ((uint32_t)t << 23);
+  const uint32_t qhi = (uint32_t)(q >> 32) + ((uint32_t)(t >> 32) << 23);
+  return ((uint64_t)qhi << 32) | qlo;
+}
+
+// Of every 8 column pairs, how many take exp2 on the FMA pipes (the rest use MUFU).
+#ifndef RESS_POLY_PAIRS_PER8
+#define RESS_POLY_PAIRS_PER8 2
+#endif
+constexpr int kPolyPairsPer8 = RESS_POLY_PAIRS_PER8;
 
 // Instruction descriptors, kind::f16: bf16 A and B, fp32 accumulator.
 //   S  = Q K^T : M = 128, N = 128, A and B K-major.
@@ -94,9 +160,13 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   if (tid == 0) {
     mbar_init(&bar->q_full, 1);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bar->kv_full[s], 1);
-      mbar_init(&bar->kv_empty[s], 1);
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(&bar->k_full[s], 1);
+      mbar_init(&bar->k_empty[s], 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(&bar->v_full[s], 1);
+      mbar_init(&bar->v_empty[s], 1);
     }
     mbar_init(&bar->s_full, 1);
     mbar_init(&bar->s_free, 4);
@@ -106,7 +176,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     bar->abort = 0;
     fence_mbar_init();
   }
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // validate the row before any work: count in range, every entry in [0, nb)
     bool bad = cnt < 0 || cnt > p.nb;
     if (!bad)
@@ -118,7 +188,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (lane == 0) bar->row_state = bad ? 2 : (cnt == 0 ? 1 : 0);
     if (bad && lane == 0) report_error(p.dev_err, RESS_ERR_DEVICE_BOUNDS);
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(&bar->tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -130,34 +200,54 @@ __global__ void __launch_bounds__(kThreads, 2)
   volatile int *abort = &bar->abort;
 
   if (state == 0) {
-    if (warp == 4) {
+    if (warp == kProducerWarp) {
       // ------------------------------------------------------------ TMA producer
+      // One thread keeps both rings full.  S_j finishes before PV_j, so the slot of K_j
+      // frees before that of V_j: waiting in that order never blocks a load that a
+      // consumer needs earlier.
       if (lane == 0) {
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
         mbar_arrive_expect_tx(&bar->q_full, kTile);
         tma_load_3d(smem + kOffQ, &tmQ, &bar->q_full, 0, qi * 128, (int)bh);
-        int issued = 0;
+        auto load_k = [&](int j) {
+          const int s = j % kKStages;
+          mbar_arrive_expect_tx(&bar->k_full[s], kTile);
+          tma_load_3d(smem + kOffK + s * kTile, &tmK, &bar->k_full[s], 0, kvrow[j] * 128, (int)bh);
+        };
+        auto load_v = [&](int j) {
+          const int s = j % kVStages;
+          mbar_arrive_expect_tx(&bar->v_full[s], kTile);
+          tma_load_3d(smem + kOffV + s * kTile, &tmV, &bar->v_full[s], 0, kvrow[j] * 128, (int)bh);
+        };
+        int nk = min(cnt, kKStages), nv = min(cnt, kVStages);
+        for (int j = 0; j < nk; ++j) load_k(j);
+        for (int j = 0; j < nv; ++j) load_v(j);
         for (int j = 0; j < cnt; ++j) {
-          const int s = j % kStages;
-          if (j >= kStages && !mbar_wait(&bar->kv_empty[s], ((j / kStages) - 1) & 1, abort)) {
-            report_error(p.dev_err, RESS_ERR_DEVICE_TIMEOUT);
-            *abort = 1;
-            break;
+          if (j + kKStages < cnt) {
+            if (!mbar_wait(&bar->k_empty[j % kKStages], (j / kKStages) & 1, abort)) break;
+            load_k(j + kKStages);
+            nk = j + kKStages + 1;
           }
-          const int kb = kvrow[j];
-          mbar_arrive_expect_tx(&bar->kv_full[s], 2 * kTile);
-          tma_load_3d(smem + kOffK + s * kTile, &tmK, &bar->kv_full[s], 0, kb * 128, (int)bh);
-          tma_load_3d(smem + kOffV + s * kTile, &tmV, &bar->kv_full[s], 0, kb * 128, (int)bh);
-          issued = j + 1;
+          if (j + kVStages < cnt) {
+            if (!mbar_wait(&bar->v_empty[j % kVStages], (j / kVStages) & 1, abort)) break;
+            load_v(j + kVStages);
+            nv = j + kVStages + 1;
+          }
+        }
+        if (*abort == 0 && (nk < cnt || nv < cnt)) {
+          report_error(p.dev_err, RESS_ERR_DEVICE_TIMEOUT);
+          *abort = 1;
         }
         // never leave the CTA with copies in flight
-        for (int j = max(0, issued - kStages); j < issued; ++j)
-          mbar_wait(&bar->kv_full[j % kStages], (j / kStages) & 1, nullptr);
+        for (int j = max(0, nk - kKStages); j < nk; ++j)
+          mbar_wait(&bar->k_full[j % kKStages], (j / kKStages) & 1, nullptr);
+        for (int j = max(0, nv - kVStages); j < nv; ++j)
+          mbar_wait(&bar->v_full[j % kVStages], (j / kVStages) & 1, nullptr);
         mbar_wait(&bar->q_full, 0, nullptr);
       }
-    } else if (warp == 5) {
+    } else if (warp == kMmaWarp) {
       // ------------------------------------------------------ tensor-core issuer
       if (lane == 0) {
         const uint32_t sQ = smem_u32(smem + kOffQ);
@@ -168,8 +258,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         const uint64_t dq = smem_desc(sQ);
         for (int j = 0; ok && j <= cnt; ++j) {
           if (j < cnt) {
-            const int s = j % kStages;
-            ok = mbar_wait(&bar->kv_full[s], (j / kStages) & 1, abort);
+            const int s = j % kKStages;
+            ok = mbar_wait(&bar->k_full[s], (j / kKStages) & 1, abort);
             if (ok && j > 0) ok = mbar_wait(&bar->s_free, (j - 1) & 1, abort);
             if (!ok) break;
             tc_fence_after();
@@ -177,10 +267,12 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
             for (int k = 0; k < 4; ++k) mma_ss(tmem + kColS, dq + 2 * k, dk + 2 * k, kIdescS, k > 0);
             mma_commit(&bar->s_full);
+            mma_commit(&bar->k_empty[s]);
           }
           if (j > 0) {
-            const int jp = j - 1, sp = jp % kStages;
+            const int jp = j - 1, sp = jp % kVStages;
             ok = mbar_wait(&bar->p_full, jp & 1, abort);
+            if (ok) ok = mbar_wait(&bar->v_full[sp], (jp / kVStages) & 1, abort);
             if (!ok) break;
             tc_fence_after();
             const uint64_t dv = smem_desc(sV + sp * kTile);
@@ -188,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             for (int k = 0; k < 8; ++k)
               mma_ts(tmem + kColO, tmem + kColP + 8 * k, dv + 128 * k, kIdescPV, (jp > 0 || k > 0));
             mma_commit(&bar->o_done);
-            mma_commit(&bar->kv_empty[sp]);
+            mma_commit(&bar->v_empty[sp]);
           }
         }
         if (!ok) {
@@ -206,42 +298,62 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int last_valid = p.N - (p.nb - 1) * 128;  // tokens in the last block
       float m_run = -INFINITY, l_run = 0.f;
       bool ok = true;
+      int kb_next = kvrow[0];
       for (int j = 0; j < cnt && ok; ++j) {
+        const int kb = kb_next;
+        if (j + 1 < cnt) kb_next = kvrow[j + 1];
         ok = mbar_wait(&bar->s_full, j & 1, abort);
         if (!ok) break;
         tc_fence_after();
         uint32_t sv[128];
-        tmem_ld32(trow + kColS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-        tmem_ld32(trow + kColS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-        tmem_ld32(trow + kColS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
-        tmem_ld32(trow + kColS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
+#pragma unroll
+        for (int h = 0; h < 4; ++h)
+          tmem_ld32(trow + kColS + 32 * h, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * h]));
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar->s_free);
-        const int kb = kvrow[j];
         if (kb == p.nb - 1 && last_valid < 128) {
 #pragma unroll
           for (int c = 0; c < 128; ++c)
             if (c >= last_valid) sv[c] = __float_as_uint(-INFINITY);
         }
-        float mx = __uint_as_float(sv[0]);
+        // row max: four chains of 3-input max
+        float mc[4];
 #pragma unroll
-        for (int c = 1; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(sv[c]));
+        for (int q = 0; q < 4; ++q) mc[q] = fmaxf(__uint_as_float(sv[2 * q]), __uint_as_float(sv[2 * q + 1]));
+#pragma unroll
+        for (int c = 8; c < 128; c += 8) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            mc[q] = fmax3(mc[q], __uint_as_float(sv[c + 2 * q]), __uint_as_float(sv[c + 2 * q + 1]));
+        }
+        const float mx = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3]));
         const float m_new = fmaxf(m_run, mx * p.scale_log2);
-        const bool rescale = m_new > m_run + 8.0f;
+        const bool rescale = m_new > m_run + kRescaleLog2;
         const float m_use = rescale ? m_new : m_run;
         const float alpha = rescale ? ex2_approx(m_run - m_new) : 1.0f;
-        float sum = 0.f;
+        // p = 2^(s * scale_log2 - m_use): packed FMA, exp2 split between MUFU and the FMA
+        // pipes, packed row sums in four chains, bf16 pairs for the P tile
+        const uint64_t sc2 = f2(p.scale_log2, p.scale_log2);
+        const uint64_t nm2 = f2(-m_use, -m_use);
+        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
         uint32_t pk[64];
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * c]), p.scale_log2, -m_use));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * c + 1]), p.scale_log2, -m_use));
-          sum += p0 + p1;
-          pk[c] = pack_bf16x2(p0, p1);
+          const uint64_t x = ffma2(f2(__uint_as_float(sv[2 * c]), __uint_as_float(sv[2 * c + 1])), sc2, nm2);
+          uint64_t e;
+          if ((c & 7) < kPolyPairsPer8) {
+            e = exp2_pair_fma(x);
+          } else {
+            e = f2(ex2_approx(f2lo(x)), ex2_approx(f2hi(x)));
+          }
+          acc[c & 3] = fadd2(acc[c & 3], e);
+          pk[c] = pack_bf16x2(f2lo(e), f2hi(e));
         }
-        l_run = l_run * alpha + sum;
+        const uint64_t a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
+        const uint64_t a = fadd2(a01, a23);
+        l_run = l_run * alpha + (f2lo(a) + f2hi(a));
         if (j > 0) {
           ok = mbar_wait(&bar->o_done, (j - 1) & 1, abort);
           if (!ok) break;
@@ -306,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) tmem_dealloc(tmem, kTmemCols);
+  if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {

@@ -230,3 +230,29 @@ def test_schedule_is_a_stable_descending_permutation():
     flat = cnt.flatten().tolist()
     want = sorted(range(48), key=lambda it: (-flat[it], it))
     assert order.cpu().tolist() == want
+
+
+def test_wide_logit_range_and_rescaling():
+    """Logits spread over hundreds of units (Q scaled by 12): exp2 arguments reach the
+    clamp at -126, the running max jumps between tiles and forces O rescales; a ragged
+    last block masks columns.  Compared with torch SDPA in fp32."""
+    ensure_built()
+    g = torch.Generator(device="cuda").manual_seed(7)
+    N = 1000
+    q = (12.0 * torch.randn(1, 2, N, 64, device="cuda", generator=g)).to(torch.bfloat16)
+    k = torch.randn(1, 2, N, 64, device="cuda", generator=g).to(torch.bfloat16)
+    v = torch.randn(1, 2, N, 64, device="cuda", generator=g).to(torch.bfloat16)
+    nb = 8
+    # every row keeps every block, in an order that makes the max grow tile by tile
+    idx = torch.arange(nb, dtype=torch.int32).expand(1, 2, nb, nb).contiguous()
+    cnt = torch.full((1, 2, nb), nb, dtype=torch.int32)
+    out = torch.empty(1, 2, N, 64, device="cuda", dtype=torch.bfloat16)
+    lse = torch.empty(1, 2, N, device="cuda")
+    R.ress_block_sparse_attn(R.make_shape(1, 2, N), q, k, v, idx.cuda(), cnt.cuda(), None, 0.125, out, lse)
+    torch.cuda.synchronize()
+    ref = torch.nn.functional.scaled_dot_product_attention(q.float(), k.float(), v.float(), scale=0.125)
+    lref = torch.logsumexp(0.125 * q.float() @ k.float().transpose(-1, -2), dim=-1)
+    assert torch.isfinite(out.float()).all()
+    assert (out.float() - ref).abs().max().item() <= 2e-2
+    assert ((out.float() - ref).norm() / ref.norm()).item() <= 1e-2
+    assert ((lse - lref).abs() <= 1e-3 + 1e-4 * lref.abs()).all()
