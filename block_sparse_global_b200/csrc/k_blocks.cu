@@ -5,6 +5,7 @@
 // Q/K/V, the block map and drift score by fp32 FMA on L2-resident pooled tensors.
 #include <cuda_bf16.h>
 
+#include "k_tiles.cuh"
 #include "ress_common.cuh"
 #include "ress_internal.h"
 
@@ -114,44 +115,51 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(const uint4 *__restrict_
 }
 
 // ---------------------------------------- pooled block map and Eq. 1 output, [ReSS] §4.1
-// One CTA per (b*h, TQ query blocks).  Logits of the CTA's rows against every key block
-// are kept in shared memory ([TQ][nb] floats), so each pooled key / value tile is read
-// once per CTA.  Warp w owns rows w, w + 8, ...
+// One CTA per (b*h, TQ query blocks); warp w owns rows w*R .. w*R+R-1 (R = TQ/8).  The
+// logits of the CTA's rows against every key block stay in shared memory ([TQ][nb]
+// floats); the head's pooled keys, then values, stream through two shared-memory tiles
+// of 64 blocks (cp.async double buffering), so each is read once per CTA.
 template <int TQ>
 __global__ void __launch_bounds__(kThreads) block_scores_kernel(
     const float *__restrict__ qp, const float *__restrict__ kp, const float *__restrict__ vp,
     float scale, float *__restrict__ P, float *__restrict__ vbar, int nb) {
+  constexpr int R = TQ / kWarps;
   extern __shared__ __align__(16) float sm[];
-  float *sq = sm;                     // [TQ][64]
-  float *st = sq + TQ * kHeadDim;     // [32][65] key or value tile
-  float *sl = st + 32 * kPad;         // [TQ][nb] logits, then probabilities
+  float *tiles = sm;                      // 2 x [64][68]
+  float *sq = tiles + 2 * kTileFloats;    // [TQ][64]
+  float *sl = sq + TQ * kHeadDim;         // [TQ][nb] logits, then probabilities
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const long long bh = blockIdx.y;
   const int i0 = blockIdx.x * TQ;
   const float *qh = qp + (size_t)bh * nb * kHeadDim;
-  const float *kh = kp + (size_t)bh * nb * kHeadDim;
-  const float *vh = vp + (size_t)bh * nb * kHeadDim;
   for (int idx = t; idx < TQ * kHeadDim; idx += kThreads) {
-    int r = idx / kHeadDim;
+    const int r = idx / kHeadDim;
     sq[idx] = (i0 + r < nb) ? qh[(size_t)(i0 + r) * kHeadDim + idx % kHeadDim] : 0.f;
   }
-  for (int j0 = 0; j0 < nb; j0 += 32) {
-    __syncthreads();
-    for (int idx = t; idx < 32 * kHeadDim; idx += kThreads) {
-      int jj = idx / kHeadDim, c = idx % kHeadDim;
-      st[jj * kPad + c] = (j0 + jj < nb) ? kh[(size_t)(j0 + jj) * kHeadDim + c] : 0.f;
+  // logits: lane takes key blocks lane and lane + 32 of each tile
+  tile_stream(tiles, kp + (size_t)bh * nb * kHeadDim, nb, [&](int tt, const float *tile) {
+    const float4 *k0 = reinterpret_cast<const float4 *>(tile + lane * kTilePad);
+    const float4 *k1 = reinterpret_cast<const float4 *>(tile + (lane + 32) * kTilePad);
+#pragma unroll
+    for (int q = 0; q < R; ++q) {
+      const int r = warp * R + q;
+      const float4 *qq = reinterpret_cast<const float4 *>(sq + r * kHeadDim);
+      float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+      for (int d = 0; d < 16; ++d) {
+        const float4 x = qq[d], y0 = k0[d], y1 = k1[d];
+        a0 = fmaf(x.x, y0.x, a0); a0 = fmaf(x.y, y0.y, a0); a0 = fmaf(x.z, y0.z, a0); a0 = fmaf(x.w, y0.w, a0);
+        a1 = fmaf(x.x, y1.x, a1); a1 = fmaf(x.y, y1.y, a1); a1 = fmaf(x.z, y1.z, a1); a1 = fmaf(x.w, y1.w, a1);
+      }
+      const int j = tt * kTileKeys + lane;
+      if (j < nb) sl[r * nb + j] = a0 * scale;
+      if (j + 32 < nb) sl[r * nb + j + 32] = a1 * scale;
     }
-    __syncthreads();
-    for (int r = warp; r < TQ; r += kWarps) {
-      float acc = 0.f;
-#pragma unroll 16
-      for (int c = 0; c < kHeadDim; ++c) acc = fmaf(sq[r * kHeadDim + c], st[lane * kPad + c], acc);
-      if (j0 + lane < nb) sl[r * nb + j0 + lane] = acc * scale;
-    }
-  }
-  __syncthreads();
-  for (int r = warp; r < TQ; r += kWarps) {
-    const int i = i0 + r;
+  });
+  // softmax over every key block, per row
+#pragma unroll
+  for (int q = 0; q < R; ++q) {
+    const int r = warp * R + q, i = i0 + r;
     if (i >= nb) continue;
     float *row = sl + r * nb;
     float m = -INFINITY;
@@ -159,48 +167,39 @@ __global__ void __launch_bounds__(kThreads) block_scores_kernel(
     m = warp_max(m);
     float sum = 0.f;
     for (int j = lane; j < nb; j += 32) {
-      float e = expf(row[j] - m);
+      const float e = expf(row[j] - m);
       row[j] = e;
       sum += e;
     }
     sum = warp_sum(sum);
     float *prow = P + ((size_t)bh * nb + i) * nb;
     for (int j = lane; j < nb; j += 32) {
-      float p = __fdiv_rn(row[j], sum);
-      row[j] = p;
-      prow[j] = p;
+      const float pj = __fdiv_rn(row[j], sum);
+      row[j] = pj;
+      prow[j] = pj;
     }
   }
-  // vbar_i = sum_j P_ij V_j, value tiles staged through shared memory.
-  float a0[(TQ + kWarps - 1) / kWarps], a1[(TQ + kWarps - 1) / kWarps];
+  // vbar_i = sum_j P_ij V_j: lane takes value dimensions lane and lane + 32
+  float a0[R], a1[R];
 #pragma unroll
-  for (int q = 0; q < (TQ + kWarps - 1) / kWarps; ++q) a0[q] = a1[q] = 0.f;
-  for (int j0 = 0; j0 < nb; j0 += 32) {
-    __syncthreads();
-    for (int idx = t; idx < 32 * kHeadDim; idx += kThreads) {
-      int jj = idx / kHeadDim, c = idx % kHeadDim;
-      st[jj * kPad + c] = (j0 + jj < nb) ? vh[(size_t)(j0 + jj) * kHeadDim + c] : 0.f;
-    }
-    __syncthreads();
-    const int jn = min(32, nb - j0);
+  for (int q = 0; q < R; ++q) a0[q] = a1[q] = 0.f;
+  tile_stream(tiles, vp + (size_t)bh * nb * kHeadDim, nb, [&](int tt, const float *tile) {
+    const int jn = min(kTileKeys, nb - tt * kTileKeys);
 #pragma unroll
-    for (int q = 0; q < (TQ + kWarps - 1) / kWarps; ++q) {
-      const int r = warp + q * kWarps;
-      if (r < TQ && i0 + r < nb) {
-        const float *row = sl + r * nb + j0;
-        for (int jj = 0; jj < jn; ++jj) {
-          const float p = row[jj];
-          a0[q] = fmaf(p, st[jj * kPad + lane], a0[q]);
-          a1[q] = fmaf(p, st[jj * kPad + lane + 32], a1[q]);
-        }
+    for (int q = 0; q < R; ++q) {
+      const float *row = sl + (warp * R + q) * nb + tt * kTileKeys;
+      for (int kk = 0; kk < jn; ++kk) {
+        const float pj = row[kk];
+        a0[q] = fmaf(pj, tile[kk * kTilePad + lane], a0[q]);
+        a1[q] = fmaf(pj, tile[kk * kTilePad + lane + 32], a1[q]);
       }
     }
-  }
+  });
 #pragma unroll
-  for (int q = 0; q < (TQ + kWarps - 1) / kWarps; ++q) {
-    const int r = warp + q * kWarps;
-    if (r < TQ && i0 + r < nb) {
-      float *o = vbar + ((size_t)bh * nb + i0 + r) * kHeadDim;
+  for (int q = 0; q < R; ++q) {
+    const int i = i0 + warp * R + q;
+    if (i < nb) {
+      float *o = vbar + ((size_t)bh * nb + i) * kHeadDim;
       o[lane] = a0[q];
       o[lane + 32] = a1[q];
     }
@@ -247,40 +246,53 @@ __global__ void __launch_bounds__(kThreads) drift_prep_kernel(
   }
 }
 
-// Pass 2: s_ij = P_ij sqrt(max(a_i - 2 w_i . V_j + c_j, 0)).  One CTA per (b*h, 8 rows);
-// lane = key within a 32-key tile staged in shared memory.
+// Pass 2: s_ij = P_ij sqrt(max(a_i - 2 w_i . V_j + c_j, 0)).  One CTA per (b*h, 16 rows),
+// two rows per warp; the head's pooled values stream through shared memory in tiles of
+// 64 blocks, lane = key block (lane and lane + 32).
+constexpr int kDriftRows = 16;
 __global__ void __launch_bounds__(kThreads) drift_kernel(
     const float *__restrict__ P, const float *__restrict__ vp, const float *__restrict__ w,
     const float *__restrict__ a, const float *__restrict__ c, float *__restrict__ s, int nb) {
-  __shared__ float sw[kWarps][kHeadDim];
-  __shared__ float sv[32][kPad];
+  constexpr int R = kDriftRows / kWarps;
+  __shared__ __align__(16) float tiles[2 * kTileFloats];
+  __shared__ __align__(16) float sw[kDriftRows][kHeadDim];
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const long long bh = blockIdx.y;
-  const int i = blockIdx.x * kWarps + warp;
-  const bool live = i < nb;
-  if (live) {
-    sw[warp][lane] = w[((size_t)bh * nb + i) * kHeadDim + lane];
-    sw[warp][lane + 32] = w[((size_t)bh * nb + i) * kHeadDim + lane + 32];
+  const int i0 = blockIdx.x * kDriftRows;
+  for (int idx = t; idx < kDriftRows * kHeadDim; idx += kThreads) {
+    const int r = idx / kHeadDim;
+    sw[r][idx % kHeadDim] = (i0 + r < nb) ? w[((size_t)bh * nb + i0 + r) * kHeadDim + idx % kHeadDim] : 0.f;
   }
-  const float ai = live ? a[(size_t)bh * nb + i] : 0.f;
-  const float *vh = vp + (size_t)bh * nb * kHeadDim;
-  for (int j0 = 0; j0 < nb; j0 += 32) {
-    __syncthreads();
-    for (int idx = t; idx < 32 * kHeadDim; idx += kThreads) {
-      int jj = idx / kHeadDim, cc = idx % kHeadDim;
-      sv[jj][cc] = (j0 + jj < nb) ? vh[(size_t)(j0 + jj) * kHeadDim + cc] : 0.f;
-    }
-    __syncthreads();
-    const int j = j0 + lane;
-    if (live && j < nb) {
-      float dot = 0.f;
-#pragma unroll 16
-      for (int e = 0; e < kHeadDim; ++e) dot = fmaf(sw[warp][e], sv[lane][e], dot);
-      const float q = (ai - 2.f * dot) + c[(size_t)bh * nb + j];
-      const size_t o = ((size_t)bh * nb + i) * nb + j;
-      s[o] = P[o] * sqrtf(fmaxf(q, 0.f));
-    }
+  float ai[R];
+#pragma unroll
+  for (int q = 0; q < R; ++q) {
+    const int i = i0 + warp * R + q;
+    ai[q] = i < nb ? a[(size_t)bh * nb + i] : 0.f;
   }
+  const float *ch = c + (size_t)bh * nb;
+  tile_stream(tiles, vp + (size_t)bh * nb * kHeadDim, nb, [&](int tt, const float *tile) {
+    const float4 *v0 = reinterpret_cast<const float4 *>(tile + lane * kTilePad);
+    const float4 *v1 = reinterpret_cast<const float4 *>(tile + (lane + 32) * kTilePad);
+    const int j0 = tt * kTileKeys + lane, j1 = j0 + 32;
+    const float c0 = j0 < nb ? ch[j0] : 0.f, c1 = j1 < nb ? ch[j1] : 0.f;
+#pragma unroll
+    for (int q = 0; q < R; ++q) {
+      const int r = warp * R + q, i = i0 + r;
+      const float4 *ww = reinterpret_cast<const float4 *>(&sw[r][0]);
+      float d0 = 0.f, d1 = 0.f;
+#pragma unroll 4
+      for (int d = 0; d < 16; ++d) {
+        const float4 x = ww[d], y0 = v0[d], y1 = v1[d];
+        d0 = fmaf(x.x, y0.x, d0); d0 = fmaf(x.y, y0.y, d0); d0 = fmaf(x.z, y0.z, d0); d0 = fmaf(x.w, y0.w, d0);
+        d1 = fmaf(x.x, y1.x, d1); d1 = fmaf(x.y, y1.y, d1); d1 = fmaf(x.z, y1.z, d1); d1 = fmaf(x.w, y1.w, d1);
+      }
+      if (i < nb) {
+        const size_t o = ((size_t)bh * nb + i) * nb;
+        if (j0 < nb) s[o + j0] = P[o + j0] * sqrtf(fmaxf((ai[q] - 2.f * d0) + c0, 0.f));
+        if (j1 < nb) s[o + j1] = P[o + j1] * sqrtf(fmaxf((ai[q] - 2.f * d1) + c1, 0.f));
+      }
+    }
+  });
 }
 
 }  // namespace
@@ -304,7 +316,7 @@ cudaError_t launch_pool(const Dims &d, const void *q, const void *k, const void 
 template <int TQ>
 static cudaError_t scores_tq(const Dims &d, const float *qp, const float *kp, const float *vp,
                              float scale, float *P, float *vbar, cudaStream_t st) {
-  const size_t smem = sizeof(float) * (TQ * kHeadDim + 32 * kPad + (size_t)TQ * d.nb);
+  const size_t smem = sizeof(float) * (2 * kTileFloats + TQ * kHeadDim + (size_t)TQ * d.nb);
   cudaError_t e = cudaFuncSetAttribute(block_scores_kernel<TQ>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -316,7 +328,7 @@ static cudaError_t scores_tq(const Dims &d, const float *qp, const float *kp, co
 cudaError_t launch_block_scores(const Dims &d, const float *qp, const float *kp, const float *vp,
                                 float scale, float *P, float *vbar, cudaStream_t st) {
   // 16 rows per CTA while their logits fit comfortably in shared memory, else 8.
-  if ((size_t)16 * d.nb * sizeof(float) <= 160 * 1024)
+  if ((size_t)16 * d.nb * sizeof(float) <= 150 * 1024)
     return scores_tq<16>(d, qp, kp, vp, scale, P, vbar, st);
   return scores_tq<8>(d, qp, kp, vp, scale, P, vbar, st);
 }
@@ -339,7 +351,7 @@ cudaError_t launch_drift(const Dims &d, const float *P, const float *vp, const f
   drift_prep_kernel<<<g1, kThreads, 0, st>>>(vp, vbar, gram, w, a, c, d.H, d.nb);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  dim3 g2((d.nb + kWarps - 1) / kWarps, (unsigned)d.BH());
+  dim3 g2((d.nb + kDriftRows - 1) / kDriftRows, (unsigned)d.BH());
   drift_kernel<<<g2, kThreads, 0, st>>>(P, vp, w, a, c, s, d.nb);
   return cudaGetLastError();
 }

@@ -1,10 +1,13 @@
 // Per-(query block, head) key-block selection and the attention launch order.
 //
 // [ReSS] = "ReSS: Residual-Restoring Sparse Attention for 3D Vision Transformers".
-// One warp owns one row (b, h, i); a CTA holds T rows of the same head so that the
-// pooled value tiles streamed through shared memory during restoration serve T rows.
-// Exact top-k is an MSB-first radix select on order-preserving integer keys (8-bit
-// digits, a shared-memory histogram per warp), ties to the lower block index.
+// One warp owns one row (b, h, i); a CTA holds up to 16 rows of the same head so that
+// the pooled value tiles streamed through shared memory during restoration (cp.async,
+// double-buffered) serve all of them.  Exact top-k is an MSB-first radix select on
+// order-preserving integer keys (8-bit digits, a shared-memory histogram per warp) that
+// finishes by ranking once the threshold bucket holds at most 32 keys; ties go to the
+// lower block index.
+#include "k_tiles.cuh"
 #include "ress_common.cuh"
 #include "ress_internal.h"
 
@@ -12,6 +15,7 @@ namespace ress {
 namespace {
 
 constexpr int kPad = 65;
+constexpr int kSelStages = 3;  // pooled-value tiles in flight during restoration
 constexpr uint8_t F_FIXED = 0;    // always-kept block (not a candidate)
 constexpr uint8_t F_KEPT = 1;     // candidate, currently kept (S)
 constexpr uint8_t F_DROP = 2;     // candidate, currently dropped (D)
@@ -49,9 +53,13 @@ RESS_DEV unsigned lanemask_lt() {
 }
 
 // Marks the k valid entries with the largest key (ties: lower index) by calling
-// mark(j).  Warp-collective.  hist: 256 words of this warp's shared memory.
+// mark(j).  Warp-collective.  MSB-first radix select with 8-bit digits over a 256-bin
+// shared-memory histogram (hist, this warp's); as soon as the bucket that holds the k-th
+// key has at most 32 members, those members are gathered (slot: 32 ints of this warp's
+// shared memory) and ranked exactly by (key descending, index ascending).
 template <typename KeyT, typename KeyFn, typename ValidFn, typename MarkFn>
-RESS_DEV void warp_top_k(int n, int k, KeyFn key, ValidFn valid, MarkFn mark, uint32_t *hist) {
+RESS_DEV void warp_top_k(int n, int k, KeyFn key, ValidFn valid, MarkFn mark, uint32_t *hist,
+                         int *slot) {
   const int lane = threadIdx.x & 31;
   int nvalid = 0;
   for (int j = lane; j < n; j += 32) nvalid += valid(j) ? 1 : 0;
@@ -65,17 +73,26 @@ RESS_DEV void warp_top_k(int n, int k, KeyFn key, ValidFn valid, MarkFn mark, ui
   }
   constexpr int BITS = sizeof(KeyT) * 8;
   KeyT prefix = 0;
-  uint32_t remaining = (uint32_t)k;
+  uint32_t remaining = (uint32_t)k, bucket = 0;
+  int shift = BITS;
 #pragma unroll 1
-  for (int shift = BITS - 8; shift >= 0; shift -= 8) {
+  while (shift > 0) {
+    const int hi_shift = shift;  // bits above the digit being resolved
+    shift -= 8;
     for (int b = lane; b < 256; b += 32) hist[b] = 0;
     __syncwarp();
-    const KeyT hi_mask = (shift + 8 >= BITS) ? KeyT(0) : (~KeyT(0) << (shift + 8));
-    for (int j = lane; j < n; j += 32) {
-      if (valid(j)) {
+    for (int base = 0; base < n; base += 32) {
+      const int j = base + lane;
+      bool in = j < n && valid(j);
+      uint32_t bin = 0;
+      if (in) {
         const KeyT kk = key(j);
-        if ((kk & hi_mask) == (prefix & hi_mask)) atomicAdd(&hist[(uint32_t)(kk >> shift) & 255u], 1u);
+        in = hi_shift >= BITS || (kk >> hi_shift) == (prefix >> hi_shift);
+        bin = (uint32_t)(kk >> shift) & 255u;
       }
+      // lanes with the same bin add once, through their lowest lane
+      const unsigned peers = __match_any_sync(0xffffffffu, in ? bin : 256u);
+      if (in && (peers & lanemask_lt()) == 0) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
     }
     __syncwarp();
     // lane l holds bins 255-8l .. 248-8l (highest digits first)
@@ -95,7 +112,7 @@ RESS_DEV void warp_top_k(int n, int k, KeyFn key, ValidFn valid, MarkFn mark, ui
     const unsigned here = __ballot_sync(0xffffffffu, excl < remaining && remaining <= incl);
     const int src = __ffs(here) - 1;
     int digit = 0;
-    uint32_t above = 0;
+    uint32_t above = 0, inbin = 0;
     if (lane == src) {
       uint32_t acc = excl;
 #pragma unroll
@@ -103,6 +120,7 @@ RESS_DEV void warp_top_k(int n, int k, KeyFn key, ValidFn valid, MarkFn mark, ui
         if (acc + cnt[q] >= remaining) {
           digit = 255 - (lane * 8 + q);
           above = acc;
+          inbin = cnt[q];
           break;
         }
         acc += cnt[q];
@@ -110,25 +128,99 @@ RESS_DEV void warp_top_k(int n, int k, KeyFn key, ValidFn valid, MarkFn mark, ui
     }
     digit = __shfl_sync(0xffffffffu, digit, src);
     above = __shfl_sync(0xffffffffu, above, src);
+    bucket = __shfl_sync(0xffffffffu, inbin, src);
     remaining -= above;
     prefix |= KeyT(digit) << shift;
     __syncwarp();
+    if (bucket <= 32) break;
   }
-  // prefix is the k-th largest key; take every larger key and the first `remaining`
-  // equal keys in ascending index order.
+  // Keys whose bits at and above `shift` exceed the bucket's are taken; the bucket's
+  // members are taken by rank.
+  const KeyT top = prefix >> shift;
   uint32_t taken = 0;
   for (int base = 0; base < n; base += 32) {
     const int j = base + lane;
     const bool v = j < n && valid(j);
-    const KeyT kk = v ? key(j) : KeyT(0);
-    const bool gt = v && kk > prefix;
-    const bool eq = v && kk == prefix;
-    const unsigned beq = __ballot_sync(0xffffffffu, eq);
-    const uint32_t rank = __popc(beq & lanemask_lt()) + taken;
-    if (gt || (eq && rank < remaining)) mark(j);
-    taken += __popc(beq);
+    const KeyT kt = v ? (key(j) >> shift) : KeyT(0);
+    if (v && kt > top) mark(j);
+    const bool inb = v && kt == top;
+    const unsigned b = __ballot_sync(0xffffffffu, inb);
+    if (bucket <= 32) {
+      if (inb) slot[taken + __popc(b & lanemask_lt())] = j;
+    } else if (inb && taken + __popc(b & lanemask_lt()) < remaining) {
+      mark(j);  // all bits resolved: the bucket holds equal keys, take the lowest indices
+    }
+    taken += __popc(b);
   }
   __syncwarp();
+  if (bucket <= 32) {
+    const bool live = lane < (int)taken;
+    const int j = live ? slot[lane] : 0;
+    const KeyT kk = live ? key(j) : KeyT(0);
+    uint32_t rank = 0;
+    for (int m = 0; m < (int)taken; ++m) {
+      const int jm = __shfl_sync(0xffffffffu, j, m);
+      const KeyT km = __shfl_sync(0xffffffffu, kk, m);
+      rank += (km > kk || (km == kk && jm < j)) ? 1u : 0u;
+    }
+    if (live && rank < remaining) mark(j);
+  }
+  __syncwarp();
+}
+
+// Marks the k valid entries with the largest key (ties: lower index) for small k by
+// repeated warp-wide arg-max: every lane keeps the best of its own entries (j = lane,
+// lane + 32, ...), the warp picks the best of the 32, its owner marks it (which makes it
+// invalid) and rescans its own entries.  Exact, and cheap while k is small.
+template <typename KeyT, typename KeyFn, typename ValidFn, typename MarkFn>
+RESS_DEV void warp_top_k_extract(int n, int k, KeyFn key, ValidFn valid, MarkFn mark) {
+  const int lane = threadIdx.x & 31;
+  auto local_best = [&](KeyT &bk, int &bj) {
+    bj = -1;
+    bk = KeyT(0);
+    for (int j = lane; j < n; j += 32) {
+      if (!valid(j)) continue;
+      const KeyT kk = key(j);
+      if (bj < 0 || kk > bk) {  // ascending scan: a tie keeps the lower index
+        bk = kk;
+        bj = j;
+      }
+    }
+  };
+  KeyT bk;
+  int bj;
+  local_best(bk, bj);
+  for (int r = 0; r < k; ++r) {
+    KeyT wk = bk;
+    int wj = bj;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const KeyT ok = __shfl_xor_sync(0xffffffffu, wk, o);
+      const int oj = __shfl_xor_sync(0xffffffffu, wj, o);
+      const bool better = oj >= 0 && (wj < 0 || ok > wk || (ok == wk && oj < wj));
+      if (better) {
+        wk = ok;
+        wj = oj;
+      }
+    }
+    if (wj < 0) break;  // fewer valid entries than k
+    if (lane == (wj & 31)) {
+      mark(wj);
+      local_best(bk, bj);
+    }
+    __syncwarp();
+  }
+  __syncwarp();
+}
+
+// Exact top-k: extraction while k is small, radix select otherwise.
+template <typename KeyT, typename KeyFn, typename ValidFn, typename MarkFn>
+RESS_DEV void warp_select(int n, int k, KeyFn key, ValidFn valid, MarkFn mark, uint32_t *hist,
+                          int *slot) {
+  if (k <= 4)
+    warp_top_k_extract<KeyT>(n, k, key, valid, mark);
+  else
+    warp_top_k<KeyT>(n, k, key, valid, mark, hist, slot);
 }
 
 // Eq. 17 swap count: max(1, round-half-up(rho c 2^-(r+1))), capped at |D| and c.
@@ -141,56 +233,54 @@ RESS_DEV int swap_count(int r, int c, float rho, int n_drop) {
 
 // Applies the chosen swaps to the net drift g (lane holds g[lane], g[lane+32]) and K
 // (Eq. 13 for restores, its mirror for drops): restores in ascending block order, then
-// drops; flags move to KEPT / DROP.
+// drops; flags move to KEPT / DROP.  The chosen blocks are first listed in `list` (this
+// warp's shared memory, room for every block), then their rows are fetched eight at a
+// time so that the loads overlap.
 RESS_DEV void apply_swaps(uint8_t *flags, int nb, const float *prow, const float *vph,
-                          float vb0, float vb1, float &g0, float &g1, float &K) {
+                          float vb0, float vb1, float &g0, float &g1, float &K, int *list) {
   const int lane = threadIdx.x & 31;
 #pragma unroll 1
   for (int pass = 0; pass < 2; ++pass) {
     const uint8_t target = pass == 0 ? F_TO_KEEP : F_TO_DROP;
+    int n = 0;
     for (int c0 = 0; c0 < nb; c0 += 32) {
       const int j = c0 + lane;
-      unsigned bal = __ballot_sync(0xffffffffu, j < nb && flags[j] == target);
-      while (bal) {
-        int kk[4];
-        int n = 0;
+      const bool sel = j < nb && flags[j] == target;
+      const unsigned bal = __ballot_sync(0xffffffffu, sel);
+      if (sel) {
+        list[n + __popc(bal & lanemask_lt())] = j;
+        flags[j] = pass == 0 ? F_KEPT : F_DROP;
+      }
+      n += __popc(bal);
+    }
+    __syncwarp();
+    for (int q0 = 0; q0 < n; q0 += 8) {
+      float pk[8], x0[8], x1[8];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          kk[q] = 0;
-          if (bal) {
-            kk[q] = c0 + __ffs(bal) - 1;
-            bal &= bal - 1;
-            ++n;
-          }
-        }
-        float pk[4], x0[4], x1[4];
+      for (int q = 0; q < 8; ++q) {
+        const int kk = q0 + q < n ? list[q0 + q] : -1;
+        pk[q] = kk >= 0 ? prow[kk] : 0.f;
+        x0[q] = kk >= 0 ? vph[(size_t)kk * kHeadDim + lane] : 0.f;
+        x1[q] = kk >= 0 ? vph[(size_t)kk * kHeadDim + lane + 32] : 0.f;
+      }
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          pk[q] = q < n ? prow[kk[q]] : 0.f;
-          x0[q] = q < n ? vph[(size_t)kk[q] * kHeadDim + lane] : 0.f;
-          x1[q] = q < n ? vph[(size_t)kk[q] * kHeadDim + lane + 32] : 0.f;
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          if (q < n) {
-            const float d0 = __fmul_rn(pk[q], __fsub_rn(vb0, x0[q]));
-            const float d1 = __fmul_rn(pk[q], __fsub_rn(vb1, x1[q]));
-            if (pass == 0) {
-              g0 = __fsub_rn(g0, d0);
-              g1 = __fsub_rn(g1, d1);
-              K = __fadd_rn(K, pk[q]);
-            } else {
-              g0 = __fadd_rn(g0, d0);
-              g1 = __fadd_rn(g1, d1);
-              K = __fsub_rn(K, pk[q]);
-            }
+      for (int q = 0; q < 8; ++q) {
+        if (q0 + q < n) {
+          const float d0 = __fmul_rn(pk[q], __fsub_rn(vb0, x0[q]));
+          const float d1 = __fmul_rn(pk[q], __fsub_rn(vb1, x1[q]));
+          if (pass == 0) {
+            g0 = __fsub_rn(g0, d0);
+            g1 = __fsub_rn(g1, d1);
+            K = __fadd_rn(K, pk[q]);
+          } else {
+            g0 = __fadd_rn(g0, d0);
+            g1 = __fadd_rn(g1, d1);
+            K = __fsub_rn(K, pk[q]);
           }
         }
       }
-      __syncwarp();
-      if (j < nb && flags[j] == target) flags[j] = pass == 0 ? F_KEPT : F_DROP;
-      __syncwarp();
     }
+    __syncwarp();
   }
 }
 
@@ -219,23 +309,33 @@ RESS_DEV float objective(float G, float K, float eps) {
   return __fdiv_rn(G, __fmul_rn(Kg, Kg));
 }
 
-__global__ void __launch_bounds__(256) select_kernel(const __grid_constant__ SelectParams p) {
+// Per-warp shared-memory block of the selection kernel: histogram, gather slots, M g,
+// then the row's gain / key array and two flag arrays (current and best drop set).
+// Rounded to 16 bytes: every warp's block starts 16-byte aligned (float4 reads of M g).
+__host__ __device__ __forceinline__ size_t select_warp_bytes(int nb) {
+  const size_t b = 1024 + 128 + 256 + 32 + (size_t)nb * 4 + 2 * (size_t)((nb + 15) & ~15);
+  return (b + 15) & ~(size_t)15;
+}
+
+__global__ void __launch_bounds__(512) select_kernel(const __grid_constant__ SelectParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int T = p.rows_per_cta, nb = p.nb;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nthreads = blockDim.x;
   const bool drift = p.method == RESS_SELECT_DRIFT;
   const bool restore = drift && p.rounds > 0;
-  // shared layout
-  float(*sM)[kPad] = reinterpret_cast<float(*)[kPad]>(smem_raw);              // 64 x 65
-  float(*sV)[kPad] = reinterpret_cast<float(*)[kPad]>(smem_raw + 64 * kPad * 4);  // 32 x 65
-  unsigned char *wbase = smem_raw + 96 * kPad * 4;
-  const size_t per_warp = 256 * 4 + 64 * 4 + (size_t)nb * 4 + 2 * (size_t)((nb + 15) & ~15);
-  unsigned char *mine = wbase + per_warp * warp;
+  // shared layout: [tiles kSelStages x 64 x 68 | M 64 x 65] (restoration only), then per warp
+  float *tiles = reinterpret_cast<float *>(smem_raw);
+  float(*sM)[kPad] = reinterpret_cast<float(*)[kPad]>(smem_raw + kSelStages * kTileFloats * 4);
+  unsigned char *wbase = smem_raw + (restore ? (kSelStages * kTileFloats + 64 * kPad) * 4 : 0);
+  unsigned char *mine = wbase + select_warp_bytes(nb) * warp;
   uint32_t *hist = reinterpret_cast<uint32_t *>(mine);
-  float *sh = reinterpret_cast<float *>(mine + 1024);
-  float *gain = reinterpret_cast<float *>(mine + 1280);
-  uint8_t *flags = mine + 1280 + (size_t)nb * 4;
+  int *slot = reinterpret_cast<int *>(mine + 1024);
+  float *sh = reinterpret_cast<float *>(mine + 1152);
+  float *scal = reinterpret_cast<float *>(mine + 1408);  // vh, G/K^2, G, K; int flag at [4]
+  float *gain = reinterpret_cast<float *>(mine + 1440);
+  int *list = reinterpret_cast<int *>(gain);  // block lists reuse the gain array
+  uint8_t *flags = mine + 1440 + (size_t)nb * 4;
   uint8_t *best = flags + ((nb + 15) & ~15);
 
   const long long bh = blockIdx.y;
@@ -267,11 +367,13 @@ __global__ void __launch_bounds__(256) select_kernel(const __grid_constant__ Sel
     auto is_cand = [&](int j) { return flags[j] == F_CAND; };
     auto keep = [&](int j) { flags[j] = F_KEPT; };
     if (p.method == RESS_SELECT_MASS) {
-      warp_top_k<uint32_t>(nb, c, [&](int j) { return float_key(prow[j]); }, is_cand, keep, hist);
+      for (int j = lane; j < nb; j += 32) gain[j] = prow[j];
+      __syncwarp();
+      warp_select<uint32_t>(nb, c, [&](int j) { return float_key(gain[j]); }, is_cand, keep, hist, slot);
     } else if (p.method == RESS_SELECT_RANDOM) {
       const uint64_t base = ((uint64_t)bh * nb + (uint64_t)i) * (uint64_t)nb;
-      warp_top_k<uint64_t>(nb, c, [&](int j) { return splitmix64_key(p.seed, base + (uint64_t)j + 1); },
-                           is_cand, keep, hist);
+      warp_select<uint64_t>(nb, c, [&](int j) { return splitmix64_key(p.seed, base + (uint64_t)j + 1); },
+                           is_cand, keep, hist, slot);
     } else {
       // Eq. 7 rank key, staged in `gain`
       for (int j = lane; j < nb; j += 32) {
@@ -279,7 +381,7 @@ __global__ void __launch_bounds__(256) select_kernel(const __grid_constant__ Sel
         gain[j] = __fdiv_rn(srow[j], fmaxf(__fsub_rn(1.f, pj), p.eps));
       }
       __syncwarp();
-      warp_top_k<uint32_t>(nb, c, [&](int j) { return float_key(gain[j]); }, is_cand, keep, hist);
+      warp_select<uint32_t>(nb, c, [&](int j) { return float_key(gain[j]); }, is_cand, keep, hist, slot);
     }
     for (int j = lane; j < nb; j += 32)
       if (flags[j] == F_CAND) flags[j] = F_DROP;
@@ -295,32 +397,49 @@ __global__ void __launch_bounds__(256) select_kernel(const __grid_constant__ Sel
       vb0 = vbr[lane];
       vb1 = vbr[lane + 32];
     }
-    // initial net drift g and kept mass K (Eq. 10), summed in ascending block order
+    // Initial net drift g and kept mass K (Eq. 10).  Gathered over whichever set is
+    // smaller: the drop set D itself (g = sum_D P_j e_j, K = 1 - sum_D P_j), or the kept
+    // blocks (always-kept and kept candidates): since vbar_i = sum over all j of P_ij V_j
+    // (Eq. 1), sum_D P_j e_j = -sum_kept P_j e_j and K = sum_kept P_j.  Ascending block
+    // order; rows are fetched eight at a time.
     float g0 = 0.f, g1 = 0.f, Psum = 0.f;
-    for (int j0 = 0; j0 < nb; j0 += 32) {
-      __syncthreads();
-      for (int idx = threadIdx.x; idx < 32 * 64; idx += nthreads) {
-        const int jj = idx >> 6, cc = idx & 63;
-        sV[jj][cc] = (j0 + jj < nb) ? vph[(size_t)(j0 + jj) * 64 + cc] : 0.f;
+    bool kept_form = false;
+    if (work) {
+      kept_form = (nb - n_drop) < n_drop;
+      int n = 0;
+      for (int c0 = 0; c0 < nb; c0 += 32) {
+        const int j = c0 + lane;
+        const bool sel = j < nb && (kept_form ? flags[j] != F_DROP : flags[j] == F_DROP);
+        const unsigned bal = __ballot_sync(0xffffffffu, sel);
+        if (sel) list[n + __popc(bal & lanemask_lt())] = j;
+        n += __popc(bal);
       }
-      __syncthreads();
-      if (work) {
-        const int j = j0 + lane;
-        const float pl = j < nb ? prow[j] : 0.f;
-        const bool dl = j < nb && flags[j] == F_DROP;
-        const unsigned bal = __ballot_sync(0xffffffffu, dl);
-        const int jn = min(32, nb - j0);
-        for (int jj = 0; jj < jn; ++jj) {
-          const float pj = __shfl_sync(0xffffffffu, pl, jj);
-          if (bal & (1u << jj)) {
-            g0 = __fadd_rn(g0, __fmul_rn(pj, __fsub_rn(vb0, sV[jj][lane])));
-            g1 = __fadd_rn(g1, __fmul_rn(pj, __fsub_rn(vb1, sV[jj][lane + 32])));
-            Psum = __fadd_rn(Psum, pj);
+      __syncwarp();
+      for (int q0 = 0; q0 < n; q0 += 8) {
+        float pk[8], x0[8], x1[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int kk = q0 + q < n ? list[q0 + q] : -1;
+          pk[q] = kk >= 0 ? prow[kk] : 0.f;
+          x0[q] = kk >= 0 ? vph[(size_t)kk * kHeadDim + lane] : 0.f;
+          x1[q] = kk >= 0 ? vph[(size_t)kk * kHeadDim + lane + 32] : 0.f;
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          if (q0 + q < n) {
+            g0 = __fadd_rn(g0, __fmul_rn(pk[q], __fsub_rn(vb0, x0[q])));
+            g1 = __fadd_rn(g1, __fmul_rn(pk[q], __fsub_rn(vb1, x1[q])));
+            Psum = __fadd_rn(Psum, pk[q]);
           }
         }
       }
+      __syncwarp();
+      if (kept_form) {
+        g0 = -g0;
+        g1 = -g1;
+      }
     }
-    float K = __fsub_rn(1.f, Psum);
+    float K = kept_form ? Psum : __fsub_rn(1.f, Psum);
     float h0 = 0.f, h1 = 0.f;
     float G = work ? gram_apply(sM, g0, g1, h0, h1) : 0.f;
     float J = objective(G, K, p.eps);
@@ -332,55 +451,116 @@ __global__ void __launch_bounds__(256) select_kernel(const __grid_constant__ Sel
 #pragma unroll 1
     for (int r = 0; r < p.rounds; ++r) {
       const int m = swap_count(r, c, p.rho, n_drop);
-      float vh = 0.f, base = 0.f;
       if (work) {
         sh[lane] = h0;
         sh[lane + 32] = h1;
-        vh = warp_sum(vb0 * h0 + vb1 * h1);
+        const float vh = warp_sum(vb0 * h0 + vb1 * h1);
         const float Kh = fmaxf(K, p.eps);
-        base = __fdiv_rn(G, __fmul_rn(Kh, Kh));
-        __syncwarp();
+        if (lane == 0) {
+          scal[0] = vh;
+          scal[1] = __fdiv_rn(G, __fmul_rn(Kh, Kh));
+          scal[2] = G;
+          scal[3] = K;
+          reinterpret_cast<int *>(scal)[4] = 1;
+        }
+      } else if (lane == 0) {
+        reinterpret_cast<int *>(scal)[4] = 0;  // no restoration work in this row
       }
-      // gains of every candidate from the start-of-round state (Eqs. 14-16)
-      for (int j0 = 0; j0 < nb; j0 += 32) {
-        __syncthreads();
-        for (int idx = threadIdx.x; idx < 32 * 64; idx += nthreads) {
-          const int jj = idx >> 6, cc = idx & 63;
-          sV[jj][cc] = (j0 + jj < nb) ? vph[(size_t)(j0 + jj) * 64 + cc] : 0.f;
-        }
-        __syncthreads();
-        const int j = j0 + lane;
-        if (work && j < nb) {
-          const uint8_t f = flags[j];
-          if (f == F_KEPT || f == F_DROP) {
-            float dot = 0.f;
-#pragma unroll 16
-            for (int e = 0; e < 64; ++e) dot = fmaf(sV[lane][e], sh[e], dot);
-            const float pj = prow[j];
-            const float sj = srow[j];
-            const float t = __fmul_rn(pj, __fsub_rn(vh, dot));  // d_j^T M g
-            const float s2 = __fmul_rn(sj, sj);
-            float dG, Kn;
-            if (f == F_DROP) {  // restore j
-              dG = __fadd_rn(__fmul_rn(-2.f, t), s2);
-              Kn = fmaxf(__fadd_rn(K, pj), p.eps);
-            } else {            // drop j
-              dG = __fadd_rn(__fmul_rn(2.f, t), s2);
-              Kn = fmaxf(__fsub_rn(K, pj), p.eps);
+      __syncwarp();
+      // Gains of every candidate from the start-of-round state (Eqs. 14-16), computed by
+      // the whole CTA: a 64-block tile is 16 groups of four blocks; warp w takes groups
+      // w, w + T, ... and lane = (row lane & 15, block pair lane >> 4), so a tile row read
+      // from shared memory serves every row of the CTA at once.
+      {
+        const int rr = lane & 15, kp = lane >> 4;
+        const bool rlive = rr < T;
+        unsigned char *rb = wbase + select_warp_bytes(nb) * (rlive ? rr : 0);
+        const float *rh = reinterpret_cast<const float *>(rb + 1152);
+        const float *rs = reinterpret_cast<const float *>(rb + 1408);
+        float *rgain = reinterpret_cast<float *>(rb + 1440);
+        const uint8_t *rflags = rb + 1440 + (size_t)nb * 4;
+        const int ri = blockIdx.x * T + rr;
+        const float *rp = p.P + ((size_t)bh * nb + (ri < nb ? ri : 0)) * nb;
+        const float *rsr = p.s + ((size_t)bh * nb + (ri < nb ? ri : 0)) * nb;
+        const bool rvalid = rlive && ri < nb;
+        // P and s of this lane's blocks, fetched one tile ahead (up to 4 block groups
+        // per warp: T >= 4 rows per CTA)
+        float pn[4][2], sn[4][2];
+        auto fetch = [&](int tt) {
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const int kg = warp + g * T;
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              const int j = tt * kTileKeys + 4 * kg + 2 * kp + q;
+              const bool ok = rvalid && kg < 16 && j < nb;
+              pn[g][q] = ok ? rp[j] : 0.f;
+              sn[g][q] = ok ? rsr[j] : 0.f;
             }
-            gain[j] = __fsub_rn(base, __fdiv_rn(__fadd_rn(G, dG), __fmul_rn(Kn, Kn)));
           }
-        }
+        };
+        fetch(0);
+        tile_stream_n<kSelStages>(tiles, vph, nb, [&](int tt, const float *tile) {
+          float pc[4][2], sc[4][2];
+#pragma unroll
+          for (int g = 0; g < 4; ++g)
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              pc[g][q] = pn[g][q];
+              sc[g][q] = sn[g][q];
+            }
+          fetch(tt + 1);
+          // the rows' flags and scalars are read only here, after the stream's barrier
+          // has made every warp's writes of this round visible
+          if (!(rlive && reinterpret_cast<const int *>(rs)[4] == 1)) return;
+          const float vh = rs[0], base = rs[1], G = rs[2], Kr = rs[3];
+          const float4 *hh = reinterpret_cast<const float4 *>(rh);
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const int kg = warp + g * T;
+            if (kg >= 16) break;
+            const int kw = 4 * kg + 2 * kp;  // this lane's two blocks within the tile
+            const int j0 = tt * kTileKeys + kw;
+            const float4 *v0 = reinterpret_cast<const float4 *>(tile + kw * kTilePad);
+            const float4 *v1 = reinterpret_cast<const float4 *>(tile + (kw + 1) * kTilePad);
+            float d0 = 0.f, d1 = 0.f;
+#pragma unroll
+            for (int d = 0; d < 16; ++d) {
+              const float4 x = hh[d], y0 = v0[d], y1 = v1[d];
+              d0 = fmaf(y0.x, x.x, d0); d0 = fmaf(y0.y, x.y, d0); d0 = fmaf(y0.z, x.z, d0); d0 = fmaf(y0.w, x.w, d0);
+              d1 = fmaf(y1.x, x.x, d1); d1 = fmaf(y1.y, x.y, d1); d1 = fmaf(y1.z, x.z, d1); d1 = fmaf(y1.w, x.w, d1);
+            }
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              const int j = j0 + q;
+              if (j >= nb) continue;
+              const uint8_t f = rflags[j];
+              if (f != F_KEPT && f != F_DROP) continue;
+              const float pj = pc[g][q], sj = sc[g][q];
+              const float t = __fmul_rn(pj, __fsub_rn(vh, q == 0 ? d0 : d1));  // d_j^T M g
+              const float s2 = __fmul_rn(sj, sj);
+              float dG, Kn;
+              if (f == F_DROP) {  // restore j
+                dG = __fadd_rn(__fmul_rn(-2.f, t), s2);
+                Kn = fmaxf(__fadd_rn(Kr, pj), p.eps);
+              } else {            // drop j
+                dG = __fadd_rn(__fmul_rn(2.f, t), s2);
+                Kn = fmaxf(__fsub_rn(Kr, pj), p.eps);
+              }
+              rgain[j] = __fsub_rn(base, __fdiv_rn(__fadd_rn(G, dG), __fmul_rn(Kn, Kn)));
+            }
+          }
+        });
       }
       if (work) {
         __syncwarp();
-        warp_top_k<uint32_t>(nb, m, [&](int j) { return float_key(gain[j]); },
+        warp_select<uint32_t>(nb, m, [&](int j) { return float_key(gain[j]); },
                              [&](int j) { return flags[j] == F_DROP; },
-                             [&](int j) { flags[j] = F_TO_KEEP; }, hist);
-        warp_top_k<uint32_t>(nb, m, [&](int j) { return float_key(gain[j]); },
+                             [&](int j) { flags[j] = F_TO_KEEP; }, hist, slot);
+        warp_select<uint32_t>(nb, m, [&](int j) { return float_key(gain[j]); },
                              [&](int j) { return flags[j] == F_KEPT; },
-                             [&](int j) { flags[j] = F_TO_DROP; }, hist);
-        apply_swaps(flags, nb, prow, vph, vb0, vb1, g0, g1, K);
+                             [&](int j) { flags[j] = F_TO_DROP; }, hist, slot);
+        apply_swaps(flags, nb, prow, vph, vb0, vb1, g0, g1, K, list);
         G = gram_apply(sM, g0, g1, h0, h1);
         J = objective(G, K, p.eps);
         if (J < bestJ) {  // track-best
@@ -458,9 +638,8 @@ __global__ void __launch_bounds__(1024) schedule_kernel(const int32_t *__restric
 
 }  // namespace
 
-static size_t select_smem(int nb, int T) {
-  const size_t per_warp = 256 * 4 + 64 * 4 + (size_t)nb * 4 + 2 * (size_t)((nb + 15) & ~15);
-  return 96 * kPad * 4 + per_warp * T;
+static size_t select_smem(int nb, int T, bool restore) {
+  return (restore ? (kSelStages * kTileFloats + 64 * kPad) * 4 : 0) + select_warp_bytes(nb) * T;
 }
 
 cudaError_t launch_select(const Dims &d, const SelectLaunch &a, cudaStream_t st) {
@@ -484,10 +663,12 @@ cudaError_t launch_select(const Dims &d, const SelectLaunch &a, cudaStream_t st)
   p.mask = a.mask;
   p.dev_err = a.dev_err;
   for (int h = 0; h < d.H; ++h) p.budgets[h] = a.budgets[h];
-  int T = 8;
-  while (T > 1 && select_smem(d.nb, T) > 200 * 1024) --T;
+  const bool restore = a.method == RESS_SELECT_DRIFT && a.rounds > 0;
+  // rows per CTA: a power of two (the cooperative gain pass maps 16 rows to lanes)
+  int T = 16;
+  while (T > 4 && select_smem(d.nb, T, restore) > 220 * 1024) T >>= 1;
   p.rows_per_cta = T;
-  const size_t smem = select_smem(d.nb, T);
+  const size_t smem = select_smem(d.nb, T, restore);
   cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
