@@ -135,6 +135,23 @@ def kept_tile_flops(kv_idx, kv_cnt, N: int) -> float:
     return float(per_row.sum().item()) * 4.0 * 64.0
 
 
+def reduce_over_ranks(ms: float, work: float) -> tuple[float, float]:
+    """Whole-job figures of a weak-scaling run: (max over ranks of the device time, sum over
+    ranks of the work).  Identity without an initialised process group; the reduction runs
+    on the backend's own device (CUDA tensors for NCCL, host tensors for gloo)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(ms), float(work)
+    dev = torch.device("cuda", torch.cuda.current_device()) if dist.get_backend() == "nccl" \
+        else torch.device("cpu")
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=dev)
+    w = torch.tensor([float(work)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(w, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(w.item())
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -207,15 +224,7 @@ def run_ours(args):
     step_ms = [e[0].elapsed_time(e[2]) for e in ev]
     attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
     total_ms = sum(step_ms)
-    t = torch.tensor([total_ms, flops * args.steps], dtype=torch.float64, device=dev)
-    if world > 1:
-        tmax = t[:1].clone()
-        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
-        fsum = t[1:].clone()
-        dist.all_reduce(fsum, op=dist.ReduceOp.SUM)
-        total_ms_max, flops_all = float(tmax.item()), float(fsum.item())
-    else:
-        total_ms_max, flops_all = total_ms, flops * args.steps
+    total_ms_max, flops_all = reduce_over_ranks(total_ms, flops * args.steps)
     value = flops_all / (total_ms_max * 1e-3) / 1e12
 
     extra = {}
@@ -284,8 +293,8 @@ def run_ours(args):
                 torch.cuda.synchronize()
                 if s >= 2:
                     e2e_ms.append(a.elapsed_time(b))
-            em = statistics.mean(e2e_ms)
-            extra["e2e"] = {"value": round(flops / (em * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+            em, e2e_flops = reduce_over_ranks(statistics.mean(e2e_ms), flops)
+            extra["e2e"] = {"value": round(e2e_flops / (em * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                             "ms_per_step": round(em, 4),
                             "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
                             "d2h_bytes_per_step": layer.out.numel() * layer.out.element_size()}
