@@ -54,6 +54,24 @@ def parse():
     return ap.parse_args()
 
 
+def measured_traffic(workload: str):
+    """DRAM bytes (read + write) of one attention launch from the committed ncu record,
+    or None when the record is for another workload or the kernel source has changed
+    since the counters were taken."""
+    import hashlib
+    rec = os.path.join(ROOT, "profiles", f"attn_kernel_{workload}_traffic.txt")
+    src = os.path.join(ROOT, "block_sparse_global_b200", "csrc", "k_attn.cu")
+    try:
+        kv = dict(l.strip().split("=", 1) for l in open(rec) if "=" in l and not l.startswith("#"))
+        with open(src, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+    except OSError:
+        return None
+    if kv.get("kernel_source_sha256") != sha or kv.get("workload") != workload:
+        return None
+    return int(kv["dram_bytes_read"]) + int(kv["dram_bytes_write"])
+
+
 def peaks():
     try:
         with open(PEAKS_FILE) as f:
@@ -324,7 +342,8 @@ def run_ours(args):
         },
         "roofline": {"kernel": "block_sparse_attn", "bound": "tensor", "achieved": round(achieved, 2),
                      "peak": bf16_peak, "unit": "TFLOP/s", "frac": round(achieved / bf16_peak, 4),
-                     "peak_source": f"{peak_kind} dense bf16 (burst)", "traffic": None,
+                     "peak_source": f"{peak_kind} dense bf16 (burst)",
+                     "traffic": measured_traffic(wl.case.name), "traffic_unit": "bytes per launch (ncu)",
                      "mean_launch_ms": round(attn_mean, 4)},
         "gpu_launches": args.steps * layer.kernel_launches(wl.method),
     }
