@@ -28,6 +28,12 @@ Readings of points the pages leave open (each is also listed in the design doc):
                     recomputed from the new g.
     random control  key(b,h,i,j) = SplitMix64 output number (linear index + 1) of a
                     generator seeded with `seed`; keep the c largest keys.
+    sign flip       the drift-maximising control of [ReSS] Fig. 8: "swap only" negates
+                    the Eq. 16 gains (each round restores and drops the moves that raise J
+                    most) and keeps the selection of largest J seen; "full" also keeps the
+                    c candidates with the SMALLEST rank key kappa in the initial selection.
+    realized drift  J of a returned selection = Eq. 12 on its drop set (Eq. 10), for any
+                    method ([ReSS] §6.1, Figs. 7 and 9); 0 for a dense query block.
 Parity status: every function below is pinned by tests/test_oracle_*.py.  The exact
 swap trajectory of the restoration is pinned only through the readings above and the
 brute-force bounds (J_opt <= J_ress <= J_init); the pages print no trajectory.
@@ -40,6 +46,7 @@ from typing import Optional, Sequence
 import numpy as np
 
 MASS, DRIFT, RANDOM = 0, 1, 2
+MINIMISE, MAXIMISE_SWAPS, MAXIMISE_FULL = 0, 1, 2   # drift objective ([ReSS] Fig. 8)
 MASK64 = (1 << 64) - 1
 SPLITMIX_GAMMA = 0x9E3779B97F4A7C15
 
@@ -217,35 +224,59 @@ def swap_gains(D, S, P_row, s_sq, v_pool_head, vbar_row, h, G, K, eps: float,
     return gain, float(base)
 
 
+def realized_drift(selected: Sequence[int], cand: Sequence[int], P_row, v_pool_head, vbar_row,
+                   M, eps: float, dtype=np.float32) -> float:
+    """Eq. 12 objective of a selection: J of its drop set D = candidates not selected
+    (Eq. 10), as [ReSS] §6.1 reports it per selection."""
+    D = set(cand) - set(selected)
+    g, K = net_drift(D, P_row, v_pool_head, vbar_row, dtype)
+    return float(objective(g, K, M, eps, dtype)[0])
+
+
 def select_row(method: int, P_row, cand: Sequence[int], budget: int, *, s_row=None,
                v_pool_head=None, vbar_row=None, M=None, rounds: int = 0, rho: float = 0.5,
-               eps: float = 1e-4, rand_keys=None, dtype=np.float32) -> dict:
+               eps: float = 1e-4, rand_keys=None, sign: int = MINIMISE,
+               dtype=np.float32) -> dict:
     """Block selection for one (query block, head) row.
+
+    `sign` selects the drift objective (drift only): MINIMISE ([ReSS] §4), or the
+    maximising controls of Fig. 8, MAXIMISE_SWAPS (restoration rounds only) and
+    MAXIMISE_FULL (initial selection too).
 
     Returns dict(selected = sorted kept candidates, margin = smallest relative decision
     gap met on the way, J_init / J_best = Eq. 12 objective of the initial and returned drop
-    sets (drift only), swaps = blocks restored over all rounds, J_trace = J after each
-    round)."""
+    sets (drift with rounds only), J = realized drift of the returned selection (when M,
+    the pooled values and vbar are given), swaps = blocks restored over all rounds,
+    J_trace = J after each round)."""
     cand = list(cand)
     c = max(0, min(budget, len(cand)))
-    out = dict(margin=math.inf, J_init=None, J_best=None, swaps=0, J_trace=[])
+    out = dict(margin=math.inf, J_init=None, J_best=None, J=None, swaps=0, J_trace=[])
+    have_state = M is not None and v_pool_head is not None and vbar_row is not None
+
+    def finish(selected, margin, J=None):
+        out.update(selected=sorted(selected), margin=margin)
+        if J is None and have_state:
+            J = realized_drift(selected, cand, P_row, v_pool_head, vbar_row, M, eps, dtype)
+        out["J"] = None if J is None else float(J)
+        return out
+
+    assert sign == MINIMISE or method == DRIFT, "the sign flip is defined for drift selection"
     if method == MASS:
         sel, mg = top_by_score(cand, {j: float(dtype(P_row[j])) for j in cand}, c)
-        out.update(selected=sorted(sel), margin=mg)
-        return out
+        return finish(sel, mg)
     if method == RANDOM:
         sel, _ = top_by_score(cand, {j: rand_keys[j] for j in cand}, c)
-        out.update(selected=sorted(sel))
-        return out
+        return finish(sel, math.inf)
     assert method == DRIFT
+    maximise = sign != MINIMISE
     P_row = np.asarray(P_row, dtype=dtype)
     kap = rank_key(P_row, s_row, eps, dtype)
-    S0, margin = top_by_score(cand, {j: float(kap[j]) for j in cand}, c)
+    flip0 = -1.0 if sign == MAXIMISE_FULL else 1.0
+    S0, margin = top_by_score(cand, {j: flip0 * float(kap[j]) for j in cand}, c)
     S = set(S0)
     D = set(cand) - S
-    if rounds <= 0 or not D:
-        out.update(selected=sorted(S), margin=margin)
-        return out
+    if rounds <= 0 or not D or c == 0:
+        return finish(S, margin)
     vbar_row = np.asarray(vbar_row, dtype=dtype)
     Vp = np.asarray(v_pool_head, dtype=dtype)
     s_sq = {j: float(dtype(dtype(s_row[j]) * dtype(s_row[j]))) for j in cand}
@@ -256,6 +287,8 @@ def select_row(method: int, P_row, cand: Sequence[int], budget: int, *, s_row=No
     for r in range(rounds):
         m = swap_count(r, c, rho, len(D))
         gain, base = swap_gains(D, S, P_row, s_sq, Vp, vbar_row, h, G, K, eps, dtype)
+        if maximise:       # the moves that raise J most ([ReSS] Fig. 8)
+            gain = {k: -v for k, v in gain.items()}
         restore, mg1 = top_by_score(sorted(D), gain, m, scale=float(base))
         drop, mg2 = top_by_score(sorted(S), gain, m, scale=float(base))
         margin = min(margin, mg1, mg2)
@@ -271,15 +304,17 @@ def select_row(method: int, P_row, cand: Sequence[int], budget: int, *, s_row=No
         J, G, h = objective(g, K, M, eps, dtype)
         out["J_trace"].append(float(J))
         margin = min(margin, _rel_gap(float(J), float(best_J)))
-        if J < best_J:       # track-best, [ReSS] §4.3 last paragraph and Supp. B.3
+        # track-best, [ReSS] §4.3 last paragraph and Supp. B.3 (track-worst when maximising)
+        if (J > best_J) if maximise else (J < best_J):
             best_D, best_J = set(D), J
-    out.update(selected=sorted(set(cand) - best_D), margin=margin, J_best=float(best_J))
-    return out
+    out["J_best"] = float(best_J)
+    return finish(set(cand) - best_D, margin, J=best_J)
 
 
 def select_blocks(method: int, P, budgets: Sequence[int], keep_k=None, dense_q=None, *,
                   s=None, v_pool=None, vbar=None, gram=None, rounds: int = 0, rho: float = 0.5,
-                  eps: float = 1e-4, seed: int = 0, rows=None, dtype=np.float32) -> dict:
+                  eps: float = 1e-4, seed: int = 0, rows=None, sign: int = MINIMISE,
+                  dtype=np.float32) -> dict:
     """Selection for every (b, h, i) row, or for the listed `rows` only.
 
     Returns dict(kept = {(b,h,i): ascending list of kept key blocks}, margin = {...},
@@ -296,7 +331,7 @@ def select_blocks(method: int, P, budgets: Sequence[int], keep_k=None, dense_q=N
         if dense_q[i]:
             kept[(b, h, i)] = list(range(nk))
             margins[(b, h, i)] = math.inf
-            info[(b, h, i)] = dict(selected=cand, margin=math.inf)
+            info[(b, h, i)] = dict(selected=cand, margin=math.inf, J=0.0)
             continue
         rk = None
         if method == RANDOM:
@@ -307,7 +342,7 @@ def select_blocks(method: int, P, budgets: Sequence[int], keep_k=None, dense_q=N
                          v_pool_head=None if v_pool is None else v_pool[b, h],
                          vbar_row=None if vbar is None else vbar[b, h, i],
                          M=None if gram is None else gram[h], rounds=rounds, rho=rho, eps=eps,
-                         rand_keys=rk, dtype=dtype)
+                         rand_keys=rk, sign=sign, dtype=dtype)
         kept[(b, h, i)] = sorted(always + res["selected"])
         margins[(b, h, i)] = res["margin"]
         info[(b, h, i)] = res

@@ -171,3 +171,83 @@ def test_random_selection_keeps_largest_keys():
         base = ((b * H + h) * nq + i) * nk
         keys = stream[base:base + nk]
         assert kept == sorted(sorted(range(nk), key=lambda j: -keys[j])[:3])
+
+
+# ----------------------------------- drift-maximising control and realized J ([ReSS] §6.1)
+def test_realized_drift_is_the_masked_output_change():
+    """Eq. 12 on a selection's drop set equals ||W_O (vtilde - vbar)||^2 recomputed from
+    the attention output with the dropped blocks masked out (Eq. 11)."""
+    for seed in range(5):
+        logits, P, Vp, vbar, W, M, s = _row(seed, nk=12)
+        cand = list(range(12))
+        for sel in ([0, 3, 5], [1, 2, 4, 7, 9, 11], [6], list(range(12))):
+            J = O.realized_drift(sel, cand, P, Vp, vbar, M, 1e-12, dtype=np.float64)
+            D = set(cand) - set(sel)
+            assert J == pytest.approx(_J_masked(logits, Vp, vbar, W, D), rel=1e-9, abs=1e-18)
+
+
+def test_full_sign_flip_keeps_the_smallest_rank_keys():
+    """Fig. 8 'full': the initial selection keeps the c candidates of smallest kappa
+    (ties to the lower block index), the mirror of Eq. 7's top-c."""
+    for seed in range(6):
+        logits, P, Vp, vbar, W, M, s = _row(seed, nk=10)
+        cand = list(range(10))
+        res = O.select_row(O.DRIFT, P, cand, 4, s_row=s, v_pool_head=Vp, vbar_row=vbar, M=M,
+                           rounds=0, sign=O.MAXIMISE_FULL, dtype=np.float64)
+        kap = O.rank_key(P, s, 1e-4, np.float64)
+        assert res["selected"] == sorted(np.argsort(kap, kind="stable")[:4].tolist())
+
+
+def test_swap_only_flip_starts_from_the_minimising_selection():
+    for seed in range(4):
+        logits, P, Vp, vbar, W, M, s = _row(seed, nk=10)
+        cand = list(range(10))
+        kw = dict(s_row=s, v_pool_head=Vp, vbar_row=vbar, M=M, rounds=0, dtype=np.float64)
+        a = O.select_row(O.DRIFT, P, cand, 4, sign=O.MINIMISE, **kw)
+        b = O.select_row(O.DRIFT, P, cand, 4, sign=O.MAXIMISE_SWAPS, **kw)
+        assert a["selected"] == b["selected"] and a["J"] == b["J"]
+
+
+@pytest.mark.parametrize("sign", [O.MINIMISE, O.MAXIMISE_SWAPS, O.MAXIMISE_FULL])
+def test_returned_selection_is_the_extreme_of_its_trace(sign):
+    """Track-best (track-worst when maximising): the returned selection's J is the
+    extreme of the initial and per-round objectives, and equals the masked-output drift
+    of that selection."""
+    for seed in range(4):
+        logits, P, Vp, vbar, W, M, s = _row(seed, nk=14)
+        cand = list(range(14))
+        res = O.select_row(O.DRIFT, P, cand, 6, s_row=s, v_pool_head=Vp, vbar_row=vbar, M=M,
+                           rounds=4, sign=sign, dtype=np.float64)
+        trace = [res["J_init"]] + res["J_trace"]
+        ext = max(trace) if sign != O.MINIMISE else min(trace)
+        assert res["J_best"] == ext and res["J"] == pytest.approx(ext, rel=1e-12)
+        D = set(cand) - set(res["selected"])
+        assert res["J"] == pytest.approx(_J_masked(logits, Vp, vbar, W, D), rel=1e-9)
+
+
+def test_maximising_control_bounded_by_brute_force():
+    """Every c-subset enumerated: the maximising control's J lies between its initial J
+    and the largest J of any subset, and above the minimising selection's J."""
+    for seed in range(5):
+        logits, P, Vp, vbar, W, M, s = _row(seed, nk=9)
+        cand, c = list(range(9)), 4
+        allJ = [_J_masked(logits, Vp, vbar, W, set(cand) - set(S))
+                for S in itertools.combinations(cand, c)]
+        kw = dict(s_row=s, v_pool_head=Vp, vbar_row=vbar, M=M, rounds=5, dtype=np.float64)
+        mx = O.select_row(O.DRIFT, P, cand, c, sign=O.MAXIMISE_FULL, **kw)
+        mn = O.select_row(O.DRIFT, P, cand, c, sign=O.MINIMISE, **kw)
+        assert mx["J_init"] - 1e-15 <= mx["J"] <= max(allJ) * (1 + 1e-9)
+        assert min(allJ) * (1 - 1e-9) <= mn["J"] <= mx["J"]
+
+
+def test_realized_drift_of_mass_and_dense_rows():
+    """Mass selection reports the J of its drop set; a dense query block reports 0."""
+    logits, P, Vp, vbar, W, M, s = _row(3, nk=8)
+    P4 = np.asarray(P)[None, None, None, :].repeat(2, axis=2)
+    res = O.select_blocks(O.MASS, P4, [3], dense_q=np.array([0, 1] + [0] * 6, np.uint8)[:2],
+                          v_pool=np.asarray(Vp)[None, None], vbar=np.asarray(vbar)[None, None, None].repeat(2, axis=2),
+                          gram=np.asarray(M)[None], dtype=np.float64)
+    kept0 = res["kept"][(0, 0, 0)]
+    assert res["info"][(0, 0, 0)]["J"] == pytest.approx(
+        _J_masked(logits, Vp, vbar, W, set(range(8)) - set(kept0)), rel=1e-9)
+    assert res["info"][(0, 0, 1)]["J"] == 0.0
