@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--case", type=int, default=2, help="synthetic case index (2 = 8 views, mass 50%%)")
     ap.add_argument("--method", choices=["mass", "drift", "random"], default=None)
     ap.add_argument("--sparsity", type=float, default=None)
+    ap.add_argument("--objective", choices=["min", "max-swaps", "max-full"], default="min",
+                    help="drift objective: the method, or a drift-maximising control (drift only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--quick", action="store_true", help="timed loop only (profiling runs)")
@@ -193,6 +195,10 @@ def run_ours(args):
     R.load()
 
     wl = build_case(args, rank)
+    objective = {"min": R.DRIFT_MINIMISE, "max-swaps": R.DRIFT_MAXIMISE_SWAPS,
+                 "max-full": R.DRIFT_MAXIMISE_FULL}[args.objective]
+    if objective != R.DRIFT_MINIMISE and wl.method != R.SELECT_DRIFT:
+        raise SystemExit("--objective max-* is a control of drift selection (use --case 3/4 or --method drift)")
     Bsz, H, N, _ = wl.q.shape
     q, k, v = wl.q, wl.k, wl.v
     keep_k, dense_q = wl.keep_k, wl.dense_q
@@ -205,7 +211,8 @@ def run_ours(args):
         layer.scores(q, k, v)
         if wl.method == R.SELECT_DRIFT:
             layer.drift()
-        layer.select(wl.method, wl.budgets, keep_k, dense_q, wl.rounds, wl.rho, wl.eps, wl.select_seed)
+        layer.select(wl.method, wl.budgets, keep_k, dense_q, wl.rounds, wl.rho, wl.eps, wl.select_seed,
+                     objective=objective)
         R.ress_attn_schedule(layer.shape, layer.kv_cnt, layer.order)
 
     def attn():
@@ -221,6 +228,13 @@ def run_ours(args):
         raise SystemExit(f"device error {layer.device_error()} during warm-up")
     flops = kept_tile_flops(layer.kv_idx, layer.kv_cnt, N)
     kept_frac = float(layer.kv_cnt.sum().item()) / (Bsz * H * layer.nb * layer.nb)
+    # realized drift J of every row's selection (one extra, untimed selection pass)
+    J = torch.zeros(Bsz, H, layer.nb, device=dev)
+    layer.select(wl.method, wl.budgets, keep_k, dense_q, wl.rounds, wl.rho, wl.eps, wl.select_seed,
+                 objective=objective, drift_out=J)
+    torch.cuda.synchronize()
+    sparse_rows = J[:, :, ~wl.dense_q.bool().to(dev)] if wl.dense_q is not None else J
+    drift_mean = float(sparse_rows.mean().item())
 
     clocks = ClockSampler(local)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
@@ -255,7 +269,7 @@ def run_ours(args):
                                                         layer.scale, layer.P, layer.v_bar),
             "drift": layer.drift,
             "select": lambda: layer.select(wl.method, wl.budgets, keep_k, dense_q, wl.rounds, wl.rho,
-                                           wl.eps, wl.select_seed),
+                                           wl.eps, wl.select_seed, objective=objective),
             "schedule": lambda: R.ress_attn_schedule(layer.shape, layer.kv_cnt, layer.order),
             "attention": attn,
         }
@@ -336,6 +350,7 @@ def run_ours(args):
             "workload": wl.case.name, "batch": Bsz, "heads": H, "seq_len": N, "head_dim": 64,
             "block": 128, "method": ["mass", "drift", "random"][wl.method], "sparsity": wl.sparsity,
             "rounds": wl.rounds, "budgets": sorted(set(wl.budgets)) if len(set(wl.budgets)) < 4 else "dirichlet",
+            "drift_objective": args.objective, "realized_drift_J_mean": float(f"{drift_mean:.6g}"),
             "kept_tile_fraction": round(kept_frac, 4), "kept_tile_gflop": round(flops / 1e9, 3),
             "selection_dtype": "f32", "l2": "flushed before every timed step (256 MiB write)",
             "parallelism": f"{world} independent layers, one per GPU" if world > 1 else "single GPU",

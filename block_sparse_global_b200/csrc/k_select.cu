@@ -25,6 +25,8 @@ constexpr uint8_t F_CAND = 5;     // candidate before the initial selection
 
 struct SelectParams {
   int H, nb, method, rounds;
+  int objective;  // ress_drift_objective
+  float *drift;   // realized J per row, or null
   float rho, eps;
   uint64_t seed;
   const uint8_t *keep_k, *dense_q;
@@ -311,10 +313,12 @@ RESS_DEV float objective(float G, float K, float eps) {
 
 // Per-warp shared-memory block of the selection kernel: histogram, gather slots, M g,
 // then the row's gain / key array and two flag arrays (current and best drop set).
-// Rounded to 16 bytes: every warp's block starts 16-byte aligned (float4 reads of M g).
+// The stride is 16 bytes past a multiple of 128: every warp's block starts 16-byte
+// aligned (float4 reads of M g), and in the cooperative gain pass, where the lanes of
+// one 8-lane phase read M g of eight different rows, those reads fall on distinct banks.
 __host__ __device__ __forceinline__ size_t select_warp_bytes(int nb) {
   const size_t b = 1024 + 128 + 256 + 32 + (size_t)nb * 4 + 2 * (size_t)((nb + 15) & ~15);
-  return (b + 15) & ~(size_t)15;
+  return ((b + 127) & ~(size_t)127) + 16;
 }
 
 __global__ void __launch_bounds__(512) select_kernel(const __grid_constant__ SelectParams p) {
@@ -324,10 +328,18 @@ __global__ void __launch_bounds__(512) select_kernel(const __grid_constant__ Sel
   const int nthreads = blockDim.x;
   const bool drift = p.method == RESS_SELECT_DRIFT;
   const bool restore = drift && p.rounds > 0;
-  // shared layout: [tiles kSelStages x 64 x 68 | M 64 x 65] (restoration only), then per warp
+  const bool want_J = p.drift != nullptr;
+  const bool state = restore || want_J;  // g, K and J are tracked
+  // maximising controls ([ReSS] Fig. 8): flip the rounds' gains, and for "full" the
+  // initial rank key too
+  const bool maximise = drift && p.objective != RESS_DRIFT_MINIMISE;
+  const bool flip_init = drift && p.objective == RESS_DRIFT_MAXIMISE_FULL;
+  // shared layout: [tiles kSelStages x 64 x 68] (restoration only), [M 64 x 65] (g, K, J
+  // tracked), then per warp
+  const size_t tile_bytes = restore ? (size_t)kSelStages * kTileFloats * 4 : 0;
   float *tiles = reinterpret_cast<float *>(smem_raw);
-  float(*sM)[kPad] = reinterpret_cast<float(*)[kPad]>(smem_raw + kSelStages * kTileFloats * 4);
-  unsigned char *wbase = smem_raw + (restore ? (kSelStages * kTileFloats + 64 * kPad) * 4 : 0);
+  float(*sM)[kPad] = reinterpret_cast<float(*)[kPad]>(smem_raw + tile_bytes);
+  unsigned char *wbase = smem_raw + tile_bytes + (state ? 64 * kPad * 4 : 0);
   unsigned char *mine = wbase + select_warp_bytes(nb) * warp;
   uint32_t *hist = reinterpret_cast<uint32_t *>(mine);
   int *slot = reinterpret_cast<int *>(mine + 1024);
@@ -348,7 +360,7 @@ __global__ void __launch_bounds__(512) select_kernel(const __grid_constant__ Sel
   const float *srow = p.s ? p.s + ((size_t)bh * nb + (row_live ? i : 0)) * nb : nullptr;
   const float *vph = p.vp ? p.vp + (size_t)bh * nb * kHeadDim : nullptr;
 
-  if (restore) {
+  if (state) {
     for (int idx = threadIdx.x; idx < 64 * 64; idx += nthreads)
       sM[idx / 64][idx % 64] = p.gram[(size_t)h * 4096 + idx];
   }
@@ -375,10 +387,12 @@ __global__ void __launch_bounds__(512) select_kernel(const __grid_constant__ Sel
       warp_select<uint64_t>(nb, c, [&](int j) { return splitmix64_key(p.seed, base + (uint64_t)j + 1); },
                            is_cand, keep, hist, slot);
     } else {
-      // Eq. 7 rank key, staged in `gain`
+      // Eq. 7 rank key, staged in `gain` (negated for the "full" maximising control:
+      // the c candidates with the smallest key are kept)
       for (int j = lane; j < nb; j += 32) {
         const float pj = prow[j];
-        gain[j] = __fdiv_rn(srow[j], fmaxf(__fsub_rn(1.f, pj), p.eps));
+        const float key = __fdiv_rn(srow[j], fmaxf(__fsub_rn(1.f, pj), p.eps));
+        gain[j] = flip_init ? -key : key;
       }
       __syncwarp();
       warp_select<uint32_t>(nb, c, [&](int j) { return float_key(gain[j]); }, is_cand, keep, hist, slot);
@@ -388,9 +402,10 @@ __global__ void __launch_bounds__(512) select_kernel(const __grid_constant__ Sel
     __syncwarp();
   }
 
-  if (restore) {
+  if (state) {
     const int n_drop = n_cand - c;
-    const bool work = active && n_drop > 0 && c > 0;
+    const bool work = restore && active && n_drop > 0 && c > 0;  // restoration rounds
+    const bool gather = active && (work || want_J);              // initial g and K
     float vb0 = 0.f, vb1 = 0.f;
     if (active) {
       const float *vbr = p.vbar + ((size_t)bh * nb + i) * kHeadDim;
@@ -404,7 +419,7 @@ __global__ void __launch_bounds__(512) select_kernel(const __grid_constant__ Sel
     // order; rows are fetched eight at a time.
     float g0 = 0.f, g1 = 0.f, Psum = 0.f;
     bool kept_form = false;
-    if (work) {
+    if (gather) {
       kept_form = (nb - n_drop) < n_drop;
       int n = 0;
       for (int c0 = 0; c0 < nb; c0 += 32) {
@@ -441,7 +456,7 @@ __global__ void __launch_bounds__(512) select_kernel(const __grid_constant__ Sel
     }
     float K = kept_form ? Psum : __fsub_rn(1.f, Psum);
     float h0 = 0.f, h1 = 0.f;
-    float G = work ? gram_apply(sM, g0, g1, h0, h1) : 0.f;
+    float G = gather ? gram_apply(sM, g0, g1, h0, h1) : 0.f;
     float J = objective(G, K, p.eps);
     float bestJ = J;
     if (work) {
@@ -554,16 +569,17 @@ __global__ void __launch_bounds__(512) select_kernel(const __grid_constant__ Sel
       }
       if (work) {
         __syncwarp();
-        warp_select<uint32_t>(nb, m, [&](int j) { return float_key(gain[j]); },
-                             [&](int j) { return flags[j] == F_DROP; },
+        // the largest gains (J decreases), or for the maximising controls the largest
+        // J increases
+        auto gkey = [&](int j) { return float_key(maximise ? -gain[j] : gain[j]); };
+        warp_select<uint32_t>(nb, m, gkey, [&](int j) { return flags[j] == F_DROP; },
                              [&](int j) { flags[j] = F_TO_KEEP; }, hist, slot);
-        warp_select<uint32_t>(nb, m, [&](int j) { return float_key(gain[j]); },
-                             [&](int j) { return flags[j] == F_KEPT; },
+        warp_select<uint32_t>(nb, m, gkey, [&](int j) { return flags[j] == F_KEPT; },
                              [&](int j) { flags[j] = F_TO_DROP; }, hist, slot);
         apply_swaps(flags, nb, prow, vph, vb0, vb1, g0, g1, K, list);
         G = gram_apply(sM, g0, g1, h0, h1);
         J = objective(G, K, p.eps);
-        if (J < bestJ) {  // track-best
+        if (maximise ? J > bestJ : J < bestJ) {  // track-best (track-worst when maximising)
           bestJ = J;
           for (int j = lane; j < nb; j += 32) best[j] = flags[j];
           __syncwarp();
@@ -574,6 +590,10 @@ __global__ void __launch_bounds__(512) select_kernel(const __grid_constant__ Sel
       for (int j = lane; j < nb; j += 32) flags[j] = best[j];
       __syncwarp();
     }
+    // realized drift of the returned selection ([ReSS] §6.1): the tracked J after the
+    // rounds, else the initial one; a dense query block drops nothing
+    if (want_J && row_live && lane == 0)
+      p.drift[(size_t)bh * nb + i] = active ? (work ? bestJ : J) : 0.f;
   }
 
   // outputs: ascending kept list, count, optional mask
@@ -638,8 +658,9 @@ __global__ void __launch_bounds__(1024) schedule_kernel(const int32_t *__restric
 
 }  // namespace
 
-static size_t select_smem(int nb, int T, bool restore) {
-  return (restore ? (kSelStages * kTileFloats + 64 * kPad) * 4 : 0) + select_warp_bytes(nb) * T;
+static size_t select_smem(int nb, int T, bool restore, bool state) {
+  return (restore ? (size_t)kSelStages * kTileFloats * 4 : 0) + (state ? 64 * kPad * 4 : 0) +
+         select_warp_bytes(nb) * T;
 }
 
 cudaError_t launch_select(const Dims &d, const SelectLaunch &a, cudaStream_t st) {
@@ -651,6 +672,8 @@ cudaError_t launch_select(const Dims &d, const SelectLaunch &a, cudaStream_t st)
   p.rho = a.rho;
   p.eps = a.eps;
   p.seed = a.seed;
+  p.objective = a.objective;
+  p.drift = a.drift;
   p.keep_k = a.keep_k;
   p.dense_q = a.dense_q;
   p.P = a.P;
@@ -664,11 +687,12 @@ cudaError_t launch_select(const Dims &d, const SelectLaunch &a, cudaStream_t st)
   p.dev_err = a.dev_err;
   for (int h = 0; h < d.H; ++h) p.budgets[h] = a.budgets[h];
   const bool restore = a.method == RESS_SELECT_DRIFT && a.rounds > 0;
+  const bool state = restore || a.drift != nullptr;
   // rows per CTA: a power of two (the cooperative gain pass maps 16 rows to lanes)
   int T = 16;
-  while (T > 4 && select_smem(d.nb, T, restore) > 220 * 1024) T >>= 1;
+  while (T > 4 && select_smem(d.nb, T, restore, state) > 220 * 1024) T >>= 1;
   p.rows_per_cta = T;
-  const size_t smem = select_smem(d.nb, T, restore);
+  const size_t smem = select_smem(d.nb, T, restore, state);
   cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;

@@ -12,7 +12,7 @@ using ress::Dims;
 
 namespace {
 
-constexpr int32_t kAbiVersion = 1;
+constexpr int32_t kAbiVersion = 2;
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -133,32 +133,41 @@ ress_status ress_select_blocks(const ress_shape *shape, const ress_select_params
     return RESS_ERR_INVALID_ARG;
   for (int h = 0; h < d.H; ++h)
     if (params->budgets[h] < 0 || params->budgets[h] > d.nb) return RESS_ERR_INVALID_ARG;
+  const int obj = params->objective;
+  if (obj != RESS_DRIFT_MINIMISE && obj != RESS_DRIFT_MAXIMISE_SWAPS && obj != RESS_DRIFT_MAXIMISE_FULL)
+    return RESS_ERR_INVALID_ARG;
+  if (obj != RESS_DRIFT_MINIMISE && m != RESS_SELECT_DRIFT) return RESS_ERR_INVALID_ARG;
+  const bool want_drift = params->drift != nullptr;
   if (m == RESS_SELECT_DRIFT) {
     if (params->rounds < 0 || params->rounds > 64) return RESS_ERR_INVALID_ARG;
-    if (!(params->eps > 0.f) || !(params->rho > 0.f) || !(params->rho <= 1.f))
-      return RESS_ERR_INVALID_ARG;
+    if (!(params->rho > 0.f) || !(params->rho <= 1.f)) return RESS_ERR_INVALID_ARG;
   }
+  if ((m == RESS_SELECT_DRIFT || want_drift) && !(params->eps > 0.f)) return RESS_ERR_INVALID_ARG;
   if (empty) return RESS_OK;
   if (!ptr_ok(P) || !ptr_ok(kv_idx) || !ptr_ok(kv_cnt)) return RESS_ERR_INVALID_ARG;
   if (mask != nullptr && !aligned16(mask)) return RESS_ERR_INVALID_ARG;
   if (dev_err != nullptr && (reinterpret_cast<uintptr_t>(dev_err) & 3u)) return RESS_ERR_INVALID_ARG;
   const bool restore = m == RESS_SELECT_DRIFT && params->rounds > 0;
+  const bool state = restore || want_drift;  // the kernel tracks g, K and J
   if (m == RESS_SELECT_DRIFT && !ptr_ok(s)) return RESS_ERR_INVALID_ARG;
-  if (restore && (!ptr_ok(v_pool) || !ptr_ok(v_bar) || !ptr_ok(gram))) return RESS_ERR_INVALID_ARG;
+  if (state && (!ptr_ok(v_pool) || !ptr_ok(v_bar) || !ptr_ok(gram))) return RESS_ERR_INVALID_ARG;
+  if (want_drift && !aligned16(params->drift)) return RESS_ERR_INVALID_ARG;
   ress::SelectLaunch a;
   a.method = m;
   a.rounds = m == RESS_SELECT_DRIFT ? params->rounds : 0;
   a.rho = params->rho;
-  a.eps = m == RESS_SELECT_DRIFT ? params->eps : 1e-4f;
+  a.eps = (m == RESS_SELECT_DRIFT || want_drift) ? params->eps : 1e-4f;
+  a.objective = obj;
+  a.drift = params->drift;
   a.seed = params->seed;
   a.budgets = params->budgets;
   a.keep_k = params->keep_k;
   a.dense_q = params->dense_q;
   a.P = P;
   a.s = m == RESS_SELECT_DRIFT ? s : nullptr;
-  a.vp = restore ? v_pool : nullptr;
-  a.vbar = restore ? v_bar : nullptr;
-  a.gram = restore ? gram : nullptr;
+  a.vp = state ? v_pool : nullptr;
+  a.vbar = state ? v_bar : nullptr;
+  a.gram = state ? gram : nullptr;
   a.kv_idx = kv_idx;
   a.kv_cnt = kv_cnt;
   a.mask = mask;

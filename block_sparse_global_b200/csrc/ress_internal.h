@@ -28,7 +28,8 @@ cudaError_t launch_drift(const Dims &d, const float *P, const float *vp, const f
                          const float *gram, float *s, void *ws, cudaStream_t st);
 
 struct SelectLaunch {
-  int method, rounds;
+  int method, rounds, objective;
+  float *drift;  // realized J per row, or null
   float rho, eps;
   uint64_t seed;
   const int32_t *budgets;  // host [H]

@@ -59,12 +59,18 @@ class SparseGlobalAttention:
                             self.workspace, stream)
 
     def select(self, method: int, budgets: Sequence[int], keep_k=None, dense_q=None, rounds: int = 0,
-               rho: float = 0.5, eps: float = 1e-4, seed: int = 0, stream=None):
-        params = R.select_params(method, budgets, keep_k, dense_q, rounds, rho, eps, seed)
+               rho: float = 0.5, eps: float = 1e-4, seed: int = 0, stream=None,
+               objective: int = R.DRIFT_MINIMISE, drift_out: Optional[torch.Tensor] = None):
+        """Block selection.  `objective` flips the sign of the drift objective (the
+        maximising controls, drift only); `drift_out` (fp32 [B,H,nb]) receives each row's
+        realized drift J."""
+        params = R.select_params(method, budgets, keep_k, dense_q, rounds, rho, eps, seed,
+                                 objective, drift_out)
         drift = method == R.SELECT_DRIFT
+        state = drift or drift_out is not None
         R.ress_select_blocks(self.shape, params, self.P, self.s if drift else None,
-                             self.v_pool if drift else None, self.v_bar if drift else None,
-                             self.gram if drift else None, self.kv_idx, self.kv_cnt, self.mask,
+                             self.v_pool if state else None, self.v_bar if state else None,
+                             self.gram if state else None, self.kv_idx, self.kv_cnt, self.mask,
                              self.dev_err, stream)
 
     def attend(self, q, k, v, stream=None, schedule: bool = True):

@@ -76,6 +76,17 @@ typedef enum {
                              control of [ReSS] §6.1, Fig. 8)                         */
 } ress_method;
 
+/* Sign of the drift objective for RESS_SELECT_DRIFT.  The maximising settings are the
+ * control experiment of [ReSS] Fig. 8 ("flip the sign of the objective, either only in the
+ * restoration stage (swap only) or from the initial selection (full)", §6.1). */
+typedef enum {
+  RESS_DRIFT_MINIMISE = 0,       /* the method: keep high-drift blocks, rounds lower J   */
+  RESS_DRIFT_MAXIMISE_SWAPS = 1, /* rounds take the moves that raise J most and return
+                                    the largest J seen (initial selection unchanged)    */
+  RESS_DRIFT_MAXIMISE_FULL = 2   /* as SWAPS, and the initial selection keeps the c_h
+                                    candidates with the SMALLEST s / max(1 - P, eps)    */
+} ress_drift_objective;
+
 typedef struct {
   int32_t batch;    /* B >= 0 */
   int32_t heads;    /* H, 1..128 */
@@ -105,9 +116,17 @@ typedef struct {
   uint64_t seed;            /* RESS_SELECT_RANDOM: key of pair (b,h,i,j) is output number
                                ((b*H + h)*nb + i)*nb + j + 1 of a SplitMix64 generator
                                seeded with `seed` (Steele, Lea, Flood, OOPSLA 2014)   */
+  int32_t objective;        /* ress_drift_objective; must be RESS_DRIFT_MINIMISE unless
+                               method is RESS_SELECT_DRIFT (else INVALID_ARG)          */
+  float *drift;             /* DEVICE fp32 [B,H,nb] output or NULL: the realized drift J
+                               of every row's final selection, Eq. 12 on its drop set
+                               (Eq. 10) with K guarded by eps, for any method ([ReSS]
+                               §6.1, Figs. 7 and 9); 0 for a dense_q row.  Needs
+                               v_pool, v_bar and gram, and eps > 0.                 */
 } ress_select_params;
 
-/* Version of this ABI (incremented on any incompatible change). */
+/* Version of this ABI (incremented on any incompatible change): 2 (ress_select_params
+ * gained `objective` and `drift`). */
 int32_t ress_abi_version(void);
 
 /* Human-readable name of a status code (static string). */
@@ -210,11 +229,14 @@ ress_status ress_drift_scores_static(const ress_shape *shape, const float *P,
  *            both chosen from the start-of-round state; g and K move by Eq. 13 and its
  *            mirror; K is guarded as max(K, eps) in Eq. 16.  The drop set with the
  *            smallest J = G / max(K, eps)^2 (Eq. 12) seen, the initial one included, is
- *            returned (track-best).
+ *            returned (track-best).  params->objective flips the sign of J in the rounds
+ *            (and, for MAXIMISE_FULL, in the initial selection); the largest J seen is
+ *            then returned.
  * Every top-k orders by (score descending, block index ascending).
  *   P       fp32 [B,H,nb,nb] (ress_block_scores).
  *   s       fp32 [B,H,nb,nb] (ress_drift_scores); required for DRIFT, else may be NULL.
- *   v_pool, v_bar, gram: required for DRIFT with rounds > 0, else may be NULL.
+ *   v_pool, v_bar, gram: required for DRIFT with rounds > 0 and whenever params->drift
+ *           is set, else may be NULL.
  *   kv_idx  int32 [B,H,nb,nb] output; kv_cnt int32 [B,H,nb] output.
  *   mask    uint8 [B,H,nb,nb] output (1 = kept) or NULL.
  *   dev_err int32 device word or NULL.

@@ -74,7 +74,8 @@ class OracleLayer:
             s[(b, h, i)] = O.drift_row(self.P[b, h, i], self.vbar[b, h, i], self.vp[b, h], self.gram[h])
         return s
 
-    def select(self, rows, method, rounds, seed, P=None, s_rows=None, vp=None, vbar=None):
+    def select(self, rows, method, rounds, seed, P=None, s_rows=None, vp=None, vbar=None,
+               sign=O.MINIMISE):
         P = self.P if P is None else P
         vp = self.vp if vp is None else vp
         vbar = self.vbar if vbar is None else vbar
@@ -86,7 +87,7 @@ class OracleLayer:
                 s_full[r] = val
         return O.select_blocks(method, P, self.wl.budgets, self.keep_k, self.dense_q, s=s_full,
                                v_pool=vp, vbar=vbar, gram=self.gram, rounds=rounds,
-                               rho=self.wl.rho, eps=self.wl.eps, seed=seed, rows=rows)
+                               rho=self.wl.rho, eps=self.wl.eps, seed=seed, rows=rows, sign=sign)
 
     def attention(self, kept, rows):
         return O.block_sparse_attn(self.q, self.k, self.v, kept, self.scale, rows=rows)
@@ -132,6 +133,33 @@ def compare_masks(gpu_kept, orc_sel, nb, what):
     assert not mism, f"{what}: {len(mism)} non-ambiguous rows differ, e.g. {mism[:3]}"
     assert agree >= 0.999, f"{what}: mask agreement {agree:.5f}"
     return dict(rows=len(rows), ambiguous=amb, agreement=agree)
+
+
+def check_realized_drift(J_gpu, gpu_kept, sel, orc: OracleLayer, what):
+    """Realized J per row against the oracle's, on rows whose kept lists agree.  Both sides
+    sum g in fp32 over a hundred-odd terms (the GPU over the drop set or, through Eq. 1,
+    the kept set): the tolerance is 1e-4 of J plus 3e-5 of the scale
+    T = (sum over the larger side of P_j |vbar - V_j|)^2 |M| / K^2, which bounds the
+    cancellation in g."""
+    checked = 0
+    for r, res in sel["info"].items():
+        if res.get("J") is None or sorted(gpu_kept[r]) != sorted(sel["kept"][r]):
+            continue
+        b, h, i = r
+        if orc.dense_q[i]:
+            assert float(J_gpu[r]) == 0.0, (what, r)
+            continue
+        P = orc.P[b, h, i].astype(np.float64)
+        e = np.linalg.norm(orc.vbar[b, h, i].astype(np.float64) - orc.vp[b, h].astype(np.float64), axis=1)
+        kept = set(sel["kept"][r])
+        drop = [j for j in range(orc.nb) if j not in kept]
+        sd = float((P[drop] * e[drop]).sum()) if drop else 0.0
+        sk = float((P[list(kept)] * e[list(kept)]).sum()) if kept else 0.0
+        K = max(1.0 - float(P[drop].sum()), orc.wl.eps)
+        T = max(sd, sk) ** 2 * float(np.linalg.norm(orc.gram[h].astype(np.float64), 2)) / K ** 2
+        close([float(J_gpu[r])], [res["J"]], 1e-4, 3e-5 * T + 1e-30, f"{what} J{r}")
+        checked += 1
+    return checked
 
 
 def check_attention(layer, orc: OracleLayer, rows):

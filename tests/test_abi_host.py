@@ -39,7 +39,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert R.ress_abi_version() == 1
+    assert R.ress_abi_version() == 2
     assert R.ress_status_string(0) == "RESS_OK"
     assert R.ress_status_string(5) == "RESS_ERR_DEVICE_TIMEOUT"
     assert R.ress_status_string(99) == "RESS_ERR_UNKNOWN"
@@ -100,6 +100,19 @@ def test_select_parameter_validation(lib):
     assert lib.ress_select_blocks(shape, ctypes.byref(p), FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE,
                                   None, None, None) == INVALID          # drift needs s
     assert lib.ress_select_blocks(shape, None, *args) == INVALID
+    # the sign flip is a drift-selection control; its value must be one of the three
+    p, keep = R.select_params(0, [4, 4], objective=1)
+    assert lib.ress_select_blocks(shape, ctypes.byref(p), *args) == INVALID
+    p, keep = R.select_params(1, [4, 4], rounds=2, objective=3)
+    assert lib.ress_select_blocks(shape, ctypes.byref(p), *args) == INVALID
+    # the realized-drift output needs the pooled values, vbar and M, and a valid eps
+    p, keep = R.select_params(0, [4, 4])
+    p.drift = FAKE   # an aligned address that validation rejects before any use
+    assert lib.ress_select_blocks(shape, ctypes.byref(p), FAKE, None, None, None, None, FAKE, FAKE,
+                                  None, None, None) == INVALID
+    p, keep = R.select_params(0, [4, 4], eps=0.0)
+    p.drift = FAKE
+    assert lib.ress_select_blocks(shape, ctypes.byref(p), *args) == INVALID
 
 
 def test_python_binding_raises(lib):

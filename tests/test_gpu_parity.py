@@ -13,8 +13,8 @@ from block_sparse_global_b200 import ress as R
 from block_sparse_global_b200 import workload as W
 from block_sparse_global_b200.pipeline import SparseGlobalAttention
 from oracle import ress_oracle as O
-from parity import (OracleLayer, check_attention, check_drift, close, compare_masks, ensure_built,
-                    run_gpu, sample_rows)
+from parity import (OracleLayer, check_attention, check_drift, check_realized_drift, close,
+                    compare_masks, ensure_built, run_gpu, sample_rows)
 
 pytestmark = pytest.mark.gpu
 METHODS = {"mass": O.MASS, "drift": O.DRIFT, "random": O.RANDOM}
@@ -102,6 +102,44 @@ def test_selection_alone_on_oracle_scores():
         stats = compare_masks(layer.kept_lists(), sel, orc.nb, f"selection-only/{method}/{rounds}")
         if method == O.RANDOM:
             assert stats["agreement"] == 1.0
+
+
+@pytest.mark.parametrize("sign", [O.MINIMISE, O.MAXIMISE_SWAPS, O.MAXIMISE_FULL])
+def test_drift_objective_and_realized_drift_on_oracle_scores(sign):
+    """The drift-maximising controls of [ReSS] Fig. 8 (swap only, full) and the realized
+    drift J of every row's selection ([ReSS] §6.1), from the oracle's own P, s, pooled
+    values and Gram, against the oracle.  With MINIMISE, J is also checked for the mass
+    and random selections."""
+    wl = W.make_workload(2, heads=4, views=6, method="drift", sparsity=0.75, rounds=5)
+    ensure_built()
+    orc = OracleLayer(wl)
+    rows = _all_rows(1, 4, orc.nb)
+    s_rows = orc.drift_rows(rows)
+    s = np.zeros_like(orc.P)
+    for r, val in s_rows.items():
+        s[r] = val
+    dev = torch.device("cuda")
+    layer = SparseGlobalAttention(1, 4, wl.q.shape[2], device=dev, with_mask=True)
+    layer.P.copy_(torch.from_numpy(orc.P))
+    layer.s.copy_(torch.from_numpy(s))
+    layer.v_pool.copy_(torch.from_numpy(orc.vp))
+    layer.v_bar.copy_(torch.from_numpy(orc.vbar))
+    layer.gram.copy_(torch.from_numpy(orc.gram))
+    J = torch.full((1, 4, orc.nb), -1.0, device=dev)
+    runs = ((O.DRIFT, 0), (O.DRIFT, 5))
+    if sign == O.MINIMISE:
+        runs = runs + ((O.MASS, 0), (O.RANDOM, 0))
+    for method, rounds in runs:
+        layer.select(method, wl.budgets, wl.keep_k.to(dev), wl.dense_q.to(dev), rounds, wl.rho,
+                     wl.eps, wl.select_seed, objective=sign, drift_out=J)
+        torch.cuda.synchronize()
+        sel = orc.select(rows, method, rounds, wl.select_seed, s_rows=s_rows, sign=sign)
+        what = f"sign {sign}/{method}/{rounds}"
+        kept = layer.kept_lists()
+        compare_masks(kept, sel, orc.nb, what)
+        J_host = J.cpu().numpy()
+        n = check_realized_drift(J_host, kept, sel, orc, what)
+        assert n >= 0.9 * len(rows), (what, n)
 
 
 def test_vggt_8view_mass50_full_layer():
