@@ -207,12 +207,17 @@ def run_ours(args):
     flush = torch.empty(L2_FLUSH_BYTES // 4, device=dev, dtype=torch.float32)
     stream = torch.cuda.current_stream()
 
+    fused = wl.method != R.SELECT_DRIFT   # block map + selection in one kernel
+
     def step():
-        layer.scores(q, k, v)
-        if wl.method == R.SELECT_DRIFT:
+        if fused:
+            layer.pool(q, k, v)
+            layer.scores_select(wl.method, wl.budgets, keep_k, dense_q, wl.select_seed)
+        else:
+            layer.scores(q, k, v)
             layer.drift()
-        layer.select(wl.method, wl.budgets, keep_k, dense_q, wl.rounds, wl.rho, wl.eps, wl.select_seed,
-                     objective=objective)
+            layer.select(wl.method, wl.budgets, keep_k, dense_q, wl.rounds, wl.rho, wl.eps,
+                         wl.select_seed, objective=objective)
         R.ress_attn_schedule(layer.shape, layer.kv_cnt, layer.order)
 
     def attn():
@@ -228,8 +233,10 @@ def run_ours(args):
         raise SystemExit(f"device error {layer.device_error()} during warm-up")
     flops = kept_tile_flops(layer.kv_idx, layer.kv_cnt, N)
     kept_frac = float(layer.kv_cnt.sum().item()) / (Bsz * H * layer.nb * layer.nb)
-    # realized drift J of every row's selection (one extra, untimed selection pass)
+    # realized drift J of every row's selection (extra, untimed passes: the block map
+    # written out, then the selection with its J output)
     J = torch.zeros(Bsz, H, layer.nb, device=dev)
+    layer.scores(q, k, v)
     layer.select(wl.method, wl.budgets, keep_k, dense_q, wl.rounds, wl.rho, wl.eps, wl.select_seed,
                  objective=objective, drift_out=J)
     torch.cuda.synchronize()
@@ -262,8 +269,11 @@ def run_ours(args):
     extra = {}
     if not args.quick:
         # per-kernel breakdown (separate pass, same inputs)
-        names = ["pool", "block_scores", "drift", "select", "schedule", "attention"]
+        names = (["pool", "scores_select", "schedule", "attention"] if fused else
+                 ["pool", "block_scores", "drift", "select", "schedule", "attention"])
         calls = {
+            "scores_select": lambda: layer.scores_select(wl.method, wl.budgets, keep_k, dense_q,
+                                                         wl.select_seed),
             "pool": lambda: R.ress_pool_blocks(layer.shape, q, k, v, layer.q_pool, layer.k_pool, layer.v_pool),
             "block_scores": lambda: R.ress_block_scores(layer.shape, layer.q_pool, layer.k_pool, layer.v_pool,
                                                         layer.scale, layer.P, layer.v_bar),

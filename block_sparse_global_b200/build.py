@@ -14,7 +14,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libress.so")
 SOURCES = ["ress_api.cu", "k_blocks.cu", "k_select.cu", "k_attn.cu"]
-HEADERS = ["ress_common.cuh", "ress_internal.h", "k_tiles.cuh"]
+HEADERS = ["ress_common.cuh", "ress_internal.h", "k_tiles.cuh", "k_topk.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

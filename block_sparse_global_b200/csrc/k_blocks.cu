@@ -6,6 +6,7 @@
 #include <cuda_bf16.h>
 
 #include "k_tiles.cuh"
+#include "k_topk.cuh"
 #include "ress_common.cuh"
 #include "ress_internal.h"
 
@@ -60,20 +61,24 @@ __global__ void __launch_bounds__(kThreads) head_gram_kernel(const float *__rest
 // --------------------------------------------------- mean pooling, [ReSS] §3 step (1)
 // One warp per (tensor, b*h, block).  Lane = (token slot ts = lane/8, 16-byte column
 // group cg = lane%8): a warp-wide load covers 4 consecutive token rows (512 contiguous
-// bytes); 32 such loads cover a 128-token block.
-__global__ void __launch_bounds__(kThreads) pool_kernel(const uint4 *__restrict__ q,
-                                                        const uint4 *__restrict__ k,
-                                                        const uint4 *__restrict__ v,
-                                                        float *__restrict__ qp,
-                                                        float *__restrict__ kp,
-                                                        float *__restrict__ vp, long long BH,
-                                                        int N, int nb) {
+// bytes); 32 such loads cover a 128-token block.  Each lane issues 16 of its loads before
+// it adds any (two halves of the block), so a warp keeps 8 KB in flight; two warps per
+// CTA spread the units over every SM.  Tokens are added in the same order as a plain
+// loop over the block would.
+constexpr int kPoolWarps = 2;
+__global__ void __launch_bounds__(kPoolWarps * 32) pool_kernel(const uint4 *__restrict__ q,
+                                                               const uint4 *__restrict__ k,
+                                                               const uint4 *__restrict__ v,
+                                                               float *__restrict__ qp,
+                                                               float *__restrict__ kp,
+                                                               float *__restrict__ vp, long long BH,
+                                                               int N, int nb) {
   const int lane = threadIdx.x & 31;
   const int cg = lane & 7, ts = lane >> 3;
   const long long per_tensor = BH * nb;
   const long long units = 3 * per_tensor;
-  for (long long u = (long long)blockIdx.x * kWarps + (threadIdx.x >> 5); u < units;
-       u += (long long)gridDim.x * kWarps) {
+  for (long long u = (long long)blockIdx.x * kPoolWarps + (threadIdx.x >> 5); u < units;
+       u += (long long)gridDim.x * kPoolWarps) {
     const int which = (int)(u / per_tensor);
     const long long rem = u - which * per_tensor;
     const long long bh = rem / nb;
@@ -84,12 +89,17 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(const uint4 *__restrict_
     float acc[8];
 #pragma unroll
     for (int c = 0; c < 8; ++c) acc[c] = 0.f;
-#pragma unroll 8
-    for (int it = 0; it < kBlock / 4; ++it) {
-      const int tok = t0 + ts + 4 * it;
-      if (tok < t1) {
-        uint4 w = __ldg(src + (size_t)tok * 8 + cg);
-        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      uint4 w[16];
+#pragma unroll
+      for (int it = 0; it < 16; ++it) {
+        const int tok = t0 + ts + 4 * (it + 16 * half);
+        w[it] = tok < t1 ? __ldg(src + (size_t)tok * 8 + cg) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int it = 0; it < 16; ++it) {
+        const uint32_t ww[4] = {w[it].x, w[it].y, w[it].z, w[it].w};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           acc[2 * c] += __uint_as_float(ww[c] << 16);
@@ -119,10 +129,31 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(const uint4 *__restrict_
 // logits of the CTA's rows against every key block stay in shared memory ([TQ][nb]
 // floats); the head's pooled keys, then values, stream through two shared-memory tiles
 // of 64 blocks (cp.async double buffering), so each is read once per CTA.
-template <int TQ>
+//
+// With SEL, the same kernel also selects: each warp takes the top-c of its rows'
+// probabilities (mass) or SplitMix64 keys (random) straight from shared memory and writes
+// the kept list, so P need not go to memory and back (the fused per-row selection; the
+// drift method keeps its separate kernels).  P and vbar are then optional outputs.
+struct FusedSelect {
+  int method, H;
+  uint64_t seed;
+  const uint8_t *keep_k, *dense_q;
+  int32_t *kv_idx, *kv_cnt;
+  uint8_t *mask;
+  int budgets[kMaxHeads];
+};
+constexpr uint8_t kCand = 0, kFixed = 1, kKept = 2;  // per-block state during selection
+
+// per-warp selection scratch: histogram, gather slots, block states
+__host__ __device__ __forceinline__ size_t fused_warp_bytes(int nb) {
+  return 1024 + 128 + (size_t)((nb + 15) & ~15);
+}
+
+template <int TQ, bool SEL>
 __global__ void __launch_bounds__(kThreads) block_scores_kernel(
     const float *__restrict__ qp, const float *__restrict__ kp, const float *__restrict__ vp,
-    float scale, float *__restrict__ P, float *__restrict__ vbar, int nb) {
+    float scale, float *__restrict__ P, float *__restrict__ vbar, int nb,
+    const __grid_constant__ FusedSelect fs) {
   constexpr int R = TQ / kWarps;
   extern __shared__ __align__(16) float sm[];
   float *tiles = sm;                      // 2 x [64][68]
@@ -172,12 +203,64 @@ __global__ void __launch_bounds__(kThreads) block_scores_kernel(
       sum += e;
     }
     sum = warp_sum(sum);
-    float *prow = P + ((size_t)bh * nb + i) * nb;
+    float *prow = P ? P + ((size_t)bh * nb + i) * nb : nullptr;
     for (int j = lane; j < nb; j += 32) {
       const float pj = __fdiv_rn(row[j], sum);
       row[j] = pj;
-      prow[j] = pj;
+      if (prow) prow[j] = pj;
     }
+  }
+  if constexpr (SEL) {
+    // ------------------------------------------------ fused mass / random selection
+    // the same decisions as the selection kernel: top-c of the candidates by P (or by
+    // the SplitMix64 key), ties to the lower block index; dense rows keep every block
+    unsigned char *wb = reinterpret_cast<unsigned char *>(sl + (size_t)TQ * nb) +
+                        fused_warp_bytes(nb) * warp;
+    uint32_t *hist = reinterpret_cast<uint32_t *>(wb);
+    int *slot = reinterpret_cast<int *>(wb + 1024);
+    uint8_t *st = wb + 1152;
+    const int h = (int)(bh % fs.H);
+#pragma unroll 1
+    for (int q = 0; q < R; ++q) {
+      const int r = warp * R + q, i = i0 + r;
+      if (i >= nb) continue;
+      const float *row = sl + r * nb;
+      const bool dense = fs.dense_q != nullptr && fs.dense_q[i] != 0;
+      int n_cand = 0;
+      for (int j = lane; j < nb; j += 32) {
+        const bool fixed = fs.keep_k != nullptr && fs.keep_k[j] != 0;
+        st[j] = fixed ? kFixed : kCand;
+        n_cand += fixed ? 0 : 1;
+      }
+      n_cand = warp_sum_i(n_cand);
+      __syncwarp();
+      const int c = min(fs.budgets[h], n_cand);
+      if (!dense) {
+        auto is_cand = [&](int j) { return st[j] == kCand; };
+        auto keep = [&](int j) { st[j] = kKept; };
+        if (fs.method == RESS_SELECT_MASS) {
+          warp_select<uint32_t>(nb, c, [&](int j) { return float_key(row[j]); }, is_cand, keep, hist, slot);
+        } else {
+          const uint64_t base = ((uint64_t)bh * nb + (uint64_t)i) * (uint64_t)nb;
+          warp_select<uint64_t>(nb, c, [&](int j) { return splitmix64_key(fs.seed, base + (uint64_t)j + 1); },
+                               is_cand, keep, hist, slot);
+        }
+      }
+      int32_t *out = fs.kv_idx + ((size_t)bh * nb + i) * nb;
+      uint8_t *mrow = fs.mask ? fs.mask + ((size_t)bh * nb + i) * nb : nullptr;
+      int total = 0;
+      for (int base = 0; base < nb; base += 32) {
+        const int j = base + lane;
+        const bool k = j < nb && (dense || st[j] != kCand);
+        const unsigned bal = __ballot_sync(0xffffffffu, k);
+        if (k) out[total + __popc(bal & lanemask_lt())] = j;
+        if (mrow && j < nb) mrow[j] = k ? 1 : 0;
+        total += __popc(bal);
+      }
+      if (lane == 0) fs.kv_cnt[(size_t)bh * nb + i] = total;
+      __syncwarp();
+    }
+    if (vbar == nullptr) return;
   }
   // vbar_i = sum_j P_ij V_j: lane takes value dimensions lane and lane + 32
   float a0[R], a1[R];
@@ -305,32 +388,58 @@ cudaError_t launch_head_gram(int H, int d_model, const float *w_o, float *gram, 
 cudaError_t launch_pool(const Dims &d, const void *q, const void *k, const void *v, float *qp,
                         float *kp, float *vp, cudaStream_t st) {
   const long long units = 3 * d.BH() * d.nb;
-  long long blocks = (units + kWarps - 1) / kWarps;
-  if (blocks > 148 * 64) blocks = 148 * 64;
-  pool_kernel<<<(unsigned)blocks, kThreads, 0, st>>>(
+  long long blocks = (units + kPoolWarps - 1) / kPoolWarps;
+  if (blocks > 148 * 256) blocks = 148 * 256;
+  pool_kernel<<<(unsigned)blocks, kPoolWarps * 32, 0, st>>>(
       static_cast<const uint4 *>(q), static_cast<const uint4 *>(k), static_cast<const uint4 *>(v),
       qp, kp, vp, d.BH(), d.N, d.nb);
   return cudaGetLastError();
 }
 
-template <int TQ>
+template <int TQ, bool SEL>
 static cudaError_t scores_tq(const Dims &d, const float *qp, const float *kp, const float *vp,
-                             float scale, float *P, float *vbar, cudaStream_t st) {
-  const size_t smem = sizeof(float) * (2 * kTileFloats + TQ * kHeadDim + (size_t)TQ * d.nb);
-  cudaError_t e = cudaFuncSetAttribute(block_scores_kernel<TQ>,
+                             float scale, float *P, float *vbar, const FusedSelect &fs,
+                             cudaStream_t st) {
+  const size_t smem = sizeof(float) * (2 * kTileFloats + TQ * kHeadDim + (size_t)TQ * d.nb) +
+                      (SEL ? fused_warp_bytes(d.nb) * kWarps : 0);
+  cudaError_t e = cudaFuncSetAttribute(block_scores_kernel<TQ, SEL>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((d.nb + TQ - 1) / TQ, (unsigned)d.BH());
-  block_scores_kernel<TQ><<<grid, kThreads, smem, st>>>(qp, kp, vp, scale, P, vbar, d.nb);
+  block_scores_kernel<TQ, SEL><<<grid, kThreads, smem, st>>>(qp, kp, vp, scale, P, vbar, d.nb, fs);
   return cudaGetLastError();
+}
+
+template <bool SEL>
+static cudaError_t scores_any(const Dims &d, const float *qp, const float *kp, const float *vp,
+                              float scale, float *P, float *vbar, const FusedSelect &fs,
+                              cudaStream_t st) {
+  // 16 rows per CTA while their logits fit comfortably in shared memory and the grid
+  // still gives every SM two CTAs (296 on a 148-SM B200), else 8.
+  const long long ctas16 = (long long)((d.nb + 15) / 16) * d.BH();
+  if ((size_t)16 * d.nb * sizeof(float) <= 150 * 1024 && ctas16 >= 2 * 148)
+    return scores_tq<16, SEL>(d, qp, kp, vp, scale, P, vbar, fs, st);
+  return scores_tq<8, SEL>(d, qp, kp, vp, scale, P, vbar, fs, st);
 }
 
 cudaError_t launch_block_scores(const Dims &d, const float *qp, const float *kp, const float *vp,
                                 float scale, float *P, float *vbar, cudaStream_t st) {
-  // 16 rows per CTA while their logits fit comfortably in shared memory, else 8.
-  if ((size_t)16 * d.nb * sizeof(float) <= 150 * 1024)
-    return scores_tq<16>(d, qp, kp, vp, scale, P, vbar, st);
-  return scores_tq<8>(d, qp, kp, vp, scale, P, vbar, st);
+  FusedSelect fs{};
+  return scores_any<false>(d, qp, kp, vp, scale, P, vbar, fs, st);
+}
+
+cudaError_t launch_scores_select(const Dims &d, const ScoresSelectLaunch &a, cudaStream_t st) {
+  FusedSelect fs{};
+  fs.method = a.method;
+  fs.H = d.H;
+  fs.seed = a.seed;
+  fs.keep_k = a.keep_k;
+  fs.dense_q = a.dense_q;
+  fs.kv_idx = a.kv_idx;
+  fs.kv_cnt = a.kv_cnt;
+  fs.mask = a.mask;
+  for (int h = 0; h < d.H; ++h) fs.budgets[h] = a.budgets[h];
+  return scores_any<true>(d, a.qp, a.kp, a.vp, a.scale, a.P, a.vbar, fs, st);
 }
 
 size_t drift_workspace_bytes(const Dims &d) {

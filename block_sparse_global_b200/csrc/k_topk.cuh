@@ -1,0 +1,193 @@
+// Warp-level exact top-k selection shared by the selection kernels of libress.so: the c
+// largest keys of a row, ties to the lower index, marked through a callback.
+#pragma once
+
+#include "ress_common.cuh"
+
+namespace ress {
+
+RESS_DEV int warp_sum_i(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+RESS_DEV unsigned lanemask_lt() {
+  unsigned m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// Marks the k valid entries with the largest key (ties: lower index) by calling
+// mark(j).  Warp-collective.  MSB-first radix select with 8-bit digits over a 256-bin
+// shared-memory histogram (hist, this warp's); as soon as the bucket that holds the k-th
+// key has at most 32 members, those members are gathered (slot: 32 ints of this warp's
+// shared memory) and ranked exactly by (key descending, index ascending).
+template <typename KeyT, typename KeyFn, typename ValidFn, typename MarkFn>
+RESS_DEV void warp_top_k(int n, int k, KeyFn key, ValidFn valid, MarkFn mark, uint32_t *hist,
+                         int *slot) {
+  const int lane = threadIdx.x & 31;
+  int nvalid = 0;
+  for (int j = lane; j < n; j += 32) nvalid += valid(j) ? 1 : 0;
+  nvalid = warp_sum_i(nvalid);
+  if (k <= 0) return;
+  if (k >= nvalid) {
+    for (int j = lane; j < n; j += 32)
+      if (valid(j)) mark(j);
+    __syncwarp();
+    return;
+  }
+  constexpr int BITS = sizeof(KeyT) * 8;
+  KeyT prefix = 0;
+  uint32_t remaining = (uint32_t)k, bucket = 0;
+  int shift = BITS;
+#pragma unroll 1
+  while (shift > 0) {
+    const int hi_shift = shift;  // bits above the digit being resolved
+    shift -= 8;
+    for (int b = lane; b < 256; b += 32) hist[b] = 0;
+    __syncwarp();
+    for (int base = 0; base < n; base += 32) {
+      const int j = base + lane;
+      bool in = j < n && valid(j);
+      uint32_t bin = 0;
+      if (in) {
+        const KeyT kk = key(j);
+        in = hi_shift >= BITS || (kk >> hi_shift) == (prefix >> hi_shift);
+        bin = (uint32_t)(kk >> shift) & 255u;
+      }
+      // lanes with the same bin add once, through their lowest lane
+      const unsigned peers = __match_any_sync(0xffffffffu, in ? bin : 256u);
+      if (in && (peers & lanemask_lt()) == 0) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+    }
+    __syncwarp();
+    // lane l holds bins 255-8l .. 248-8l (highest digits first)
+    uint32_t cnt[8], tot = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      cnt[q] = hist[255 - (lane * 8 + q)];
+      tot += cnt[q];
+    }
+    uint32_t incl = tot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const uint32_t excl = incl - tot;
+    const unsigned here = __ballot_sync(0xffffffffu, excl < remaining && remaining <= incl);
+    const int src = __ffs(here) - 1;
+    int digit = 0;
+    uint32_t above = 0, inbin = 0;
+    if (lane == src) {
+      uint32_t acc = excl;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (acc + cnt[q] >= remaining) {
+          digit = 255 - (lane * 8 + q);
+          above = acc;
+          inbin = cnt[q];
+          break;
+        }
+        acc += cnt[q];
+      }
+    }
+    digit = __shfl_sync(0xffffffffu, digit, src);
+    above = __shfl_sync(0xffffffffu, above, src);
+    bucket = __shfl_sync(0xffffffffu, inbin, src);
+    remaining -= above;
+    prefix |= KeyT(digit) << shift;
+    __syncwarp();
+    if (bucket <= 32) break;
+  }
+  // Keys whose bits at and above `shift` exceed the bucket's are taken; the bucket's
+  // members are taken by rank.
+  const KeyT top = prefix >> shift;
+  uint32_t taken = 0;
+  for (int base = 0; base < n; base += 32) {
+    const int j = base + lane;
+    const bool v = j < n && valid(j);
+    const KeyT kt = v ? (key(j) >> shift) : KeyT(0);
+    if (v && kt > top) mark(j);
+    const bool inb = v && kt == top;
+    const unsigned b = __ballot_sync(0xffffffffu, inb);
+    if (bucket <= 32) {
+      if (inb) slot[taken + __popc(b & lanemask_lt())] = j;
+    } else if (inb && taken + __popc(b & lanemask_lt()) < remaining) {
+      mark(j);  // all bits resolved: the bucket holds equal keys, take the lowest indices
+    }
+    taken += __popc(b);
+  }
+  __syncwarp();
+  if (bucket <= 32) {
+    const bool live = lane < (int)taken;
+    const int j = live ? slot[lane] : 0;
+    const KeyT kk = live ? key(j) : KeyT(0);
+    uint32_t rank = 0;
+    for (int m = 0; m < (int)taken; ++m) {
+      const int jm = __shfl_sync(0xffffffffu, j, m);
+      const KeyT km = __shfl_sync(0xffffffffu, kk, m);
+      rank += (km > kk || (km == kk && jm < j)) ? 1u : 0u;
+    }
+    if (live && rank < remaining) mark(j);
+  }
+  __syncwarp();
+}
+
+// Marks the k valid entries with the largest key (ties: lower index) for small k by
+// repeated warp-wide arg-max: every lane keeps the best of its own entries (j = lane,
+// lane + 32, ...), the warp picks the best of the 32, its owner marks it (which makes it
+// invalid) and rescans its own entries.  Exact, and cheap while k is small.
+template <typename KeyT, typename KeyFn, typename ValidFn, typename MarkFn>
+RESS_DEV void warp_top_k_extract(int n, int k, KeyFn key, ValidFn valid, MarkFn mark) {
+  const int lane = threadIdx.x & 31;
+  auto local_best = [&](KeyT &bk, int &bj) {
+    bj = -1;
+    bk = KeyT(0);
+    for (int j = lane; j < n; j += 32) {
+      if (!valid(j)) continue;
+      const KeyT kk = key(j);
+      if (bj < 0 || kk > bk) {  // ascending scan: a tie keeps the lower index
+        bk = kk;
+        bj = j;
+      }
+    }
+  };
+  KeyT bk;
+  int bj;
+  local_best(bk, bj);
+  for (int r = 0; r < k; ++r) {
+    KeyT wk = bk;
+    int wj = bj;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const KeyT ok = __shfl_xor_sync(0xffffffffu, wk, o);
+      const int oj = __shfl_xor_sync(0xffffffffu, wj, o);
+      const bool better = oj >= 0 && (wj < 0 || ok > wk || (ok == wk && oj < wj));
+      if (better) {
+        wk = ok;
+        wj = oj;
+      }
+    }
+    if (wj < 0) break;  // fewer valid entries than k
+    if (lane == (wj & 31)) {
+      mark(wj);
+      local_best(bk, bj);
+    }
+    __syncwarp();
+  }
+  __syncwarp();
+}
+
+// Exact top-k: extraction while k is small, radix select otherwise.
+template <typename KeyT, typename KeyFn, typename ValidFn, typename MarkFn>
+RESS_DEV void warp_select(int n, int k, KeyFn key, ValidFn valid, MarkFn mark, uint32_t *hist,
+                          int *slot) {
+  if (k <= 4)
+    warp_top_k_extract<KeyT>(n, k, key, valid, mark);
+  else
+    warp_top_k<KeyT>(n, k, key, valid, mark, hist, slot);
+}
+
+// Eq. 17 swap count: max(1, round-half-up(rho c 2^-(r+1))), capped at |D| and c.
+
+}  // namespace ress

@@ -175,6 +175,47 @@ ress_status ress_select_blocks(const ress_shape *shape, const ress_select_params
   return from_cuda(ress::launch_select(d, a, (cudaStream_t)stream));
 }
 
+ress_status ress_scores_select(const ress_shape *shape, const ress_select_params *params,
+                               const float *q_pool, const float *k_pool, const float *v_pool,
+                               float scale, float *P, float *v_bar, int32_t *kv_idx,
+                               int32_t *kv_cnt, uint8_t *mask, int32_t *dev_err,
+                               ress_stream_t stream) {
+  Dims d;
+  bool empty;
+  ress_status st = check_shape(shape, &d, &empty);
+  if (st != RESS_OK) return st;
+  if (params == nullptr || params->budgets == nullptr) return RESS_ERR_INVALID_ARG;
+  const int m = params->method;
+  if (m == RESS_SELECT_DRIFT) return RESS_ERR_UNSUPPORTED;
+  if (m != RESS_SELECT_MASS && m != RESS_SELECT_RANDOM) return RESS_ERR_INVALID_ARG;
+  if (params->objective != RESS_DRIFT_MINIMISE || params->drift != nullptr) return RESS_ERR_INVALID_ARG;
+  for (int h = 0; h < d.H; ++h)
+    if (params->budgets[h] < 0 || params->budgets[h] > d.nb) return RESS_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || scale != scale) return RESS_ERR_INVALID_ARG;
+  if (empty) return RESS_OK;
+  if (!ptr_ok(q_pool) || !ptr_ok(k_pool) || !ptr_ok(kv_idx) || !ptr_ok(kv_cnt)) return RESS_ERR_INVALID_ARG;
+  if (P != nullptr && !aligned16(P)) return RESS_ERR_INVALID_ARG;
+  if (v_bar != nullptr && (!aligned16(v_bar) || !ptr_ok(v_pool))) return RESS_ERR_INVALID_ARG;
+  if (mask != nullptr && !aligned16(mask)) return RESS_ERR_INVALID_ARG;
+  if (dev_err != nullptr && (reinterpret_cast<uintptr_t>(dev_err) & 3u)) return RESS_ERR_INVALID_ARG;
+  ress::ScoresSelectLaunch a;
+  a.method = m;
+  a.seed = params->seed;
+  a.budgets = params->budgets;
+  a.keep_k = params->keep_k;
+  a.dense_q = params->dense_q;
+  a.qp = q_pool;
+  a.kp = k_pool;
+  a.vp = v_bar ? v_pool : nullptr;
+  a.scale = scale;
+  a.P = P;
+  a.vbar = v_bar;
+  a.kv_idx = kv_idx;
+  a.kv_cnt = kv_cnt;
+  a.mask = mask;
+  return from_cuda(ress::launch_scores_select(d, a, (cudaStream_t)stream));
+}
+
 ress_status ress_attn_schedule(const ress_shape *shape, const int32_t *kv_cnt, int32_t *work_order,
                                ress_stream_t stream) {
   Dims d;

@@ -23,6 +23,20 @@ cudaError_t launch_pool(const Dims &d, const void *q, const void *k, const void 
 cudaError_t launch_block_scores(const Dims &d, const float *qp, const float *kp, const float *vp,
                                 float scale, float *P, float *vbar, cudaStream_t st);
 
+// Block map fused with mass / random selection (P and vbar optional).
+struct ScoresSelectLaunch {
+  int method;
+  uint64_t seed;
+  const int32_t *budgets;  // host [H]
+  const uint8_t *keep_k, *dense_q;
+  const float *qp, *kp, *vp;
+  float scale;
+  float *P, *vbar;
+  int32_t *kv_idx, *kv_cnt;
+  uint8_t *mask;
+};
+cudaError_t launch_scores_select(const Dims &d, const ScoresSelectLaunch &a, cudaStream_t st);
+
 size_t drift_workspace_bytes(const Dims &d);
 cudaError_t launch_drift(const Dims &d, const float *P, const float *vp, const float *vbar,
                          const float *gram, float *s, void *ws, cudaStream_t st);

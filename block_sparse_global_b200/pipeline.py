@@ -49,10 +49,24 @@ class SparseGlobalAttention:
         R.ress_head_gram(self.shape, w_o.contiguous().float(), self.gram, stream)
 
     # ------------------------------------------------------------------ the path
-    def scores(self, q, k, v, stream=None):
+    def pool(self, q, k, v, stream=None):
         R.ress_pool_blocks(self.shape, q, k, v, self.q_pool, self.k_pool, self.v_pool, stream)
+
+    def scores(self, q, k, v, stream=None):
+        self.pool(q, k, v, stream)
         R.ress_block_scores(self.shape, self.q_pool, self.k_pool, self.v_pool, self.scale, self.P,
                             self.v_bar, stream)
+
+    def scores_select(self, method: int, budgets: Sequence[int], keep_k=None, dense_q=None,
+                      seed: int = 0, write_scores: bool = False, stream=None):
+        """Block map and MASS / RANDOM selection in one kernel (after pool()).  P and v_bar
+        are written only with write_scores."""
+        params = R.select_params(method, budgets, keep_k, dense_q, 0, 0.5, 1e-4, seed)
+        R.ress_scores_select(self.shape, params, self.q_pool, self.k_pool,
+                             self.v_pool if write_scores else None, self.scale,
+                             self.P if write_scores else None,
+                             self.v_bar if write_scores else None, self.kv_idx, self.kv_cnt,
+                             self.mask, self.dev_err, stream)
 
     def drift(self, stream=None):
         R.ress_drift_scores(self.shape, self.P, self.v_pool, self.v_bar, self.gram, self.s,
@@ -82,17 +96,21 @@ class SparseGlobalAttention:
 
     def forward(self, q, k, v, method: int, budgets: Sequence[int], keep_k=None, dense_q=None,
                 rounds: int = 0, rho: float = 0.5, eps: float = 1e-4, seed: int = 0, stream=None):
-        self.scores(q, k, v, stream)
         if method == R.SELECT_DRIFT:
+            self.scores(q, k, v, stream)
             self.drift(stream)
-        self.select(method, budgets, keep_k, dense_q, rounds, rho, eps, seed, stream)
+            self.select(method, budgets, keep_k, dense_q, rounds, rho, eps, seed, stream)
+        else:   # the block map and the selection fused in one kernel
+            self.pool(q, k, v, stream)
+            self.scores_select(method, budgets, keep_k, dense_q, seed, stream=stream)
         self.attend(q, k, v, stream)
         return self.out
 
     def kernel_launches(self, method: int) -> int:
-        """Kernels one forward() launches: pool, scores, [drift prep + drift], select,
-        schedule, attention."""
-        return 7 if method == R.SELECT_DRIFT else 5
+        """Kernels one forward() launches: drift: pool, scores, drift prep, drift, select,
+        schedule, attention; mass / random: pool, fused scores + select, schedule,
+        attention."""
+        return 7 if method == R.SELECT_DRIFT else 4
 
     def device_error(self) -> int:
         return int(self.dev_err[0].item())

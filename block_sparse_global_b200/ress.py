@@ -59,6 +59,9 @@ _SIGS = {
     "ress_drift_scores_static": (_I32, [ctypes.POINTER(ress_shape), _VP, _VP, _VP, _VP, _VP, _VP]),
     "ress_select_blocks": (_I32, [ctypes.POINTER(ress_shape), ctypes.POINTER(ress_select_params),
                                   _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
+    "ress_scores_select": (_I32, [ctypes.POINTER(ress_shape), ctypes.POINTER(ress_select_params),
+                                  _VP, _VP, _VP, ctypes.c_float, _VP, _VP, _VP, _VP, _VP, _VP,
+                                  _VP]),
     "ress_attn_schedule": (_I32, [ctypes.POINTER(ress_shape), _VP, _VP, _VP]),
     "ress_block_sparse_attn": (_I32, [ctypes.POINTER(ress_shape), _VP, _VP, _VP, _VP, _VP, _VP,
                                       ctypes.c_float, _VP, _VP, _VP, _VP]),
@@ -184,6 +187,20 @@ def ress_select_blocks(shape, params, P, s, v_pool, v_bar, gram, kv_idx, kv_cnt,
                                    _ptr(kv_cnt), _ptr(mask), _ptr(dev_err), _stream(stream))
     del keep
     _check("ress_select_blocks", st)
+
+
+def ress_scores_select(shape, params, q_pool, k_pool, v_pool, scale: float, P, v_bar, kv_idx,
+                       kv_cnt, mask=None, dev_err=None, stream=None):
+    """Block map fused with MASS / RANDOM selection; P and v_bar may be None."""
+    keep = None
+    if isinstance(params, tuple):
+        params, keep = params
+    st = load().ress_scores_select(ctypes.byref(_shape(shape)), ctypes.byref(params), _ptr(q_pool),
+                                   _ptr(k_pool), _ptr(v_pool), float(scale), _ptr(P), _ptr(v_bar),
+                                   _ptr(kv_idx), _ptr(kv_cnt), _ptr(mask), _ptr(dev_err),
+                                   _stream(stream))
+    del keep
+    _check("ress_scores_select", st)
 
 
 def ress_attn_schedule(shape, kv_cnt, work_order, stream=None):

@@ -248,6 +248,26 @@ ress_status ress_select_blocks(const ress_shape *shape, const ress_select_params
                                ress_stream_t stream);
 
 /*
+ * ress_scores_select -- ress_block_scores and ress_select_blocks in one kernel for the
+ * MASS and RANDOM methods (the fused per-row selection: each row's block map stays in
+ * shared memory from its softmax to its top-c, [ReSS] §4.3 "Fused kernel
+ * implementation" on the fusion motive).  The kept lists are identical to those of the
+ * two separate calls on the same pooled inputs.
+ *   params   as for ress_select_blocks; method must be MASS or RANDOM (else
+ *            UNSUPPORTED: drift selection needs the drift score and restoration of
+ *            its own calls), objective MINIMISE and drift NULL (else INVALID_ARG).
+ *   q_pool, k_pool  fp32 [B,H,nb,64] (ress_pool_blocks); v_pool needed only with v_bar.
+ *   P        fp32 [B,H,nb,nb] output or NULL (not written).
+ *   v_bar    fp32 [B,H,nb,64] output or NULL (Eq. 1 output not computed).
+ *   kv_idx, kv_cnt, mask, dev_err: as for ress_select_blocks.
+ */
+ress_status ress_scores_select(const ress_shape *shape, const ress_select_params *params,
+                               const float *q_pool, const float *k_pool, const float *v_pool,
+                               float scale, float *P, float *v_bar, int32_t *kv_idx,
+                               int32_t *kv_cnt, uint8_t *mask, int32_t *dev_err,
+                               ress_stream_t stream);
+
+/*
  * ress_attn_schedule -- launch order for ress_block_sparse_attn: a permutation of the
  * B*H*nb (batch, head, query block) work items sorted by kv_cnt descending, ties in
  * ascending item order (item = (b*H + h)*nb + i).  Running the longest rows first keeps

@@ -44,6 +44,11 @@ def run_gpu(wl, method=None, rounds=None, with_mask=True, seed=None):
     layer.load_output_projection(wl.w_o.to(dev))
     layer.forward(q, k, v, method, wl.budgets, wl.keep_k.to(dev), wl.dense_q.to(dev), rounds,
                   wl.rho, wl.eps, wl.select_seed if seed is None else seed)
+    if method != O.DRIFT:
+        # forward() fuses the block map into the mass / random selection and does not
+        # write P or v_bar; compute them for the checks (identical values: see
+        # test_fused_scores_select_equals_separate_calls)
+        layer.scores(q, k, v)
     torch.cuda.synchronize()
     assert layer.device_error() == 0, f"device error {layer.device_error()}"
     return layer

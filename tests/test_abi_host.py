@@ -115,6 +115,26 @@ def test_select_parameter_validation(lib):
     assert lib.ress_select_blocks(shape, ctypes.byref(p), *args) == INVALID
 
 
+def test_fused_scores_select_validation(lib):
+    shape = ctypes.byref(R.make_shape(1, 2, 1024))
+    args = [FAKE, FAKE, FAKE, 0.125, None, None, FAKE, FAKE, None, None, None]
+    p, keep = R.select_params(1, [4, 4])
+    assert lib.ress_scores_select(shape, ctypes.byref(p), *args) == UNSUPPORTED   # drift
+    p, keep = R.select_params(0, [4, 4], objective=1)
+    assert lib.ress_scores_select(shape, ctypes.byref(p), *args) == INVALID
+    p, keep = R.select_params(0, [4, 9])
+    assert lib.ress_scores_select(shape, ctypes.byref(p), *args) == INVALID       # budget > nb
+    p, keep = R.select_params(2, [4, 4])
+    assert lib.ress_scores_select(shape, ctypes.byref(p), None, *args[1:]) == INVALID
+    # v_bar requested without the pooled values
+    assert lib.ress_scores_select(shape, ctypes.byref(p), FAKE, FAKE, None, 0.125, None, FAKE,
+                                  FAKE, FAKE, None, None, None) == INVALID
+    assert lib.ress_scores_select(shape, ctypes.byref(p), FAKE, FAKE, FAKE, 0.0, None, None,
+                                  FAKE, FAKE, None, None, None) == INVALID    # scale
+    assert lib.ress_scores_select(ctypes.byref(R.make_shape(0, 2, 1024)), ctypes.byref(p),
+                                  *([None] * 3), 0.125, *([None] * 7)) == OK
+
+
 def test_python_binding_raises(lib):
     with pytest.raises(R.RessError) as e:
         R.ress_attn_schedule(R.make_shape(1, 4, 1024, head_dim=32), None, None)

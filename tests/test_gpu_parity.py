@@ -104,6 +104,36 @@ def test_selection_alone_on_oracle_scores():
             assert stats["agreement"] == 1.0
 
 
+@pytest.mark.parametrize("method", [O.MASS, O.RANDOM])
+@pytest.mark.parametrize("case", [1, 2])
+def test_fused_scores_select_equals_separate_calls(case, method):
+    """ress_scores_select (block map and selection in one kernel) against
+    ress_block_scores + ress_select_blocks on the same pooled inputs: identical kept
+    lists, counts and masks, and identical P and v_bar when it writes them."""
+    ensure_built()
+    wl = W.make_workload(case, device="cuda", heads=4, views=6) if case == 2 else W.make_workload(1, device="cuda")
+    B, H, N, _ = wl.q.shape
+    dev = torch.device("cuda")
+    ref = SparseGlobalAttention(B, H, N, device=dev, with_mask=True)
+    ref.scores(wl.q, wl.k, wl.v)
+    ref.select(method, wl.budgets, wl.keep_k, wl.dense_q, 0, wl.rho, wl.eps, wl.select_seed)
+    for write in (False, True):
+        fz = SparseGlobalAttention(B, H, N, device=dev, with_mask=True)
+        fz.pool(wl.q, wl.k, wl.v)
+        fz.P.fill_(-1.0)
+        fz.v_bar.fill_(-1.0)
+        fz.scores_select(method, wl.budgets, wl.keep_k, wl.dense_q, wl.select_seed, write_scores=write)
+        torch.cuda.synchronize()
+        assert torch.equal(fz.kv_cnt, ref.kv_cnt)
+        assert torch.equal(fz.mask, ref.mask)
+        for (b, h, i), lst in ref.kept_lists().items():
+            assert fz.kept_lists()[(b, h, i)] == lst
+        if write:
+            assert torch.equal(fz.P, ref.P) and torch.equal(fz.v_bar, ref.v_bar)
+        else:
+            assert bool((fz.P == -1.0).all()) and bool((fz.v_bar == -1.0).all())
+
+
 @pytest.mark.parametrize("sign", [O.MINIMISE, O.MAXIMISE_SWAPS, O.MAXIMISE_FULL])
 def test_drift_objective_and_realized_drift_on_oracle_scores(sign):
     """The drift-maximising controls of [ReSS] Fig. 8 (swap only, full) and the realized
