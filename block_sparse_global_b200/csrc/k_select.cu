@@ -474,6 +474,71 @@ __global__ void __launch_bounds__(1024) schedule_kernel(const int32_t *__restric
   }
 }
 
+// The same sort with the scatter spread over all 32 warps: warp w takes the contiguous
+// items [w*chunk, (w+1)*chunk), counts them per count value, a scan over the warps gives
+// each warp its first position per count value, and each warp then places its items in
+// order.  Stable and deterministic like the single-warp version; needs 32 * (nb + 1)
+// counters of shared memory.
+__global__ void __launch_bounds__(1024) schedule_kernel_par(const int32_t *__restrict__ kv_cnt,
+                                                            int32_t *__restrict__ order,
+                                                            long long items, int nb) {
+  extern __shared__ int wcnt[];  // [32][nb + 1]; row 32 of extra space: bucket starts
+  int *start = wcnt + 32 * (nb + 1);
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const long long chunk = (items + 31) / 32;
+  const long long lo = warp * chunk, hi = min(items, lo + chunk);
+  for (int i = t; i < 33 * (nb + 1); i += blockDim.x) wcnt[i] = 0;
+  __syncthreads();
+  int *mine = wcnt + warp * (nb + 1);
+  for (long long base = lo; base < hi; base += 32) {
+    const long long it = base + lane;
+    const int cv = it < hi ? min(max(kv_cnt[it], 0), nb) : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, cv);
+    if (cv >= 0 && (peers & lanemask_lt()) == 0) mine[cv] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  // bucket starts: count values largest first
+  if (warp == 0) {
+    int running = 0;
+    for (int base = 0; base <= nb; base += 32) {
+      const int c = nb - (base + lane);
+      int v = 0;
+      if (c >= 0)
+        for (int w = 0; w < 32; ++w) v += wcnt[w * (nb + 1) + c];
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (c >= 0) start[c] = running + incl - v;
+      running += __shfl_sync(0xffffffffu, incl, 31);
+    }
+  }
+  __syncthreads();
+  // per warp: its first position for every count value (exclusive scan over the warps)
+  for (int c = t; c <= nb; c += blockDim.x) {
+    int pos = start[c];
+    for (int w = 0; w < 32; ++w) {
+      const int n = wcnt[w * (nb + 1) + c];
+      wcnt[w * (nb + 1) + c] = pos;
+      pos += n;
+    }
+  }
+  __syncthreads();
+  for (long long base = lo; base < hi; base += 32) {
+    const long long it = base + lane;
+    const int cv = it < hi ? min(max(kv_cnt[it], 0), nb) : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, cv);
+    const int rank = __popc(peers & lanemask_lt());
+    if (cv >= 0) order[mine[cv] + rank] = (int32_t)it;
+    __syncwarp();
+    if (cv >= 0 && rank == 0) mine[cv] += __popc(peers);
+    __syncwarp();
+  }
+}
+
 }  // namespace
 
 static size_t select_smem(int nb, int T, bool restore, bool state) {
@@ -522,6 +587,14 @@ cudaError_t launch_select(const Dims &d, const SelectLaunch &a, cudaStream_t st)
 }
 
 cudaError_t launch_schedule(const Dims &d, const int32_t *kv_cnt, int32_t *order, cudaStream_t st) {
+  const size_t par_smem = sizeof(int) * 33 * (size_t)(d.nb + 1);
+  if (par_smem <= 200 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(schedule_kernel_par,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)par_smem);
+    if (e != cudaSuccess) return e;
+    schedule_kernel_par<<<1, 1024, par_smem, st>>>(kv_cnt, order, d.BH() * d.nb, d.nb);
+    return cudaGetLastError();
+  }
   const size_t smem = sizeof(int) * (d.nb + 1);
   cudaError_t e = cudaFuncSetAttribute(schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);

@@ -300,6 +300,23 @@ def test_schedule_is_a_stable_descending_permutation():
     assert order.cpu().tolist() == want
 
 
+def test_schedule_many_rows_and_repeated_counts():
+    """384 rows spread over the 32 warps of the parallel scatter, few distinct counts
+    (every bucket spans several warps' chunks), plus counts outside [0, nb]."""
+    ensure_built()
+    g = torch.Generator().manual_seed(5)
+    shape = R.make_shape(1, 4, 96 * 128)   # nb = 96, 384 rows
+    cnt = torch.randint(40, 44, (1, 4, 96), generator=g, dtype=torch.int32)
+    cnt[0, 1, 7] = 96
+    cnt[0, 2, 3] = -5
+    cnt[0, 3, 90] = 200
+    order = torch.empty(384, dtype=torch.int32, device="cuda")
+    R.ress_attn_schedule(shape, cnt.cuda(), order)
+    torch.cuda.synchronize()
+    flat = [min(max(c, 0), 96) for c in cnt.flatten().tolist()]
+    assert order.cpu().tolist() == sorted(range(384), key=lambda it: (-flat[it], it))
+
+
 def test_wide_logit_range_and_rescaling():
     """Logits spread over hundreds of units (Q scaled by 12): exp2 arguments reach the
     clamp at -126, the running max jumps between tiles and forces O rescales; a ragged
