@@ -106,6 +106,64 @@ class SparseGlobalAttention:
         self.attend(q, k, v, stream)
         return self.out
 
+    # ------------------------------------------------ end to end from host buffers
+    def make_groups(self, w_o: torch.Tensor, groups: int):
+        """Splits the heads into `groups` contiguous ranges for forward_host(): one layer
+        object per range, with its slice of W_O (head h owns columns 64h .. 64h+63)."""
+        if self.B != 1:
+            raise ValueError("forward_host splits heads of one batch element (B = 1)")
+        groups = max(1, min(groups, self.H))
+        bounds = [self.H * g // groups for g in range(groups + 1)]
+        self._groups = []
+        for g in range(groups):
+            h0, h1 = bounds[g], bounds[g + 1]
+            sub = SparseGlobalAttention(1, h1 - h0, self.N, device=self.device)
+            sub.load_output_projection(w_o[:, 64 * h0:64 * h1])
+            self._groups.append((h0, h1, sub))
+        self._streams = [torch.cuda.Stream(self.device) for _ in range(3)]
+        return self._groups
+
+    def forward_host(self, q_host, k_host, v_host, out_host, method: int, budgets: Sequence[int],
+                     keep_k=None, dense_q=None, rounds: int = 0, rho: float = 0.5,
+                     eps: float = 1e-4, seed: int = 0, q_dev=None, k_dev=None, v_dev=None):
+        """The layer end to end from pinned host tensors [1,H,N,64] bf16 to the pinned host
+        output.  Heads are processed in the groups of make_groups(): the copy in of group
+        g+1, the kernels of group g and the copy out of group g-1 run on three streams and
+        overlap.  RANDOM selection runs as one group (its keys depend on the head index
+        within the call).  The caller's current stream waits for the whole layer.
+        q_dev, k_dev, v_dev: optional device staging tensors of the same shape."""
+        groups = getattr(self, "_groups", None)
+        if not groups:
+            raise RuntimeError("call make_groups() first")
+        if method == R.SELECT_RANDOM and len(groups) > 1:
+            raise ValueError("random selection runs as one group")
+        q_dev = torch.empty_like(q_host, device=self.device) if q_dev is None else q_dev
+        k_dev = torch.empty_like(k_host, device=self.device) if k_dev is None else k_dev
+        v_dev = torch.empty_like(v_host, device=self.device) if v_dev is None else v_dev
+        s_in, s_cmp, s_out = self._streams
+        main = torch.cuda.current_stream(self.device)
+        for s in (s_in, s_cmp, s_out):
+            s.wait_stream(main)
+        for (h0, h1, sub) in groups:
+            with torch.cuda.stream(s_in):
+                for dev, host in ((q_dev, q_host), (k_dev, k_host), (v_dev, v_host)):
+                    dev[:, h0:h1].copy_(host[:, h0:h1], non_blocking=True)
+                arrived = torch.cuda.Event()
+                arrived.record(s_in)
+            s_cmp.wait_event(arrived)
+            with torch.cuda.stream(s_cmp):
+                sub.forward(q_dev[:, h0:h1], k_dev[:, h0:h1], v_dev[:, h0:h1], method,
+                            list(budgets)[h0:h1], keep_k, dense_q, rounds, rho, eps, seed,
+                            stream=s_cmp)
+                done = torch.cuda.Event()
+                done.record(s_cmp)
+            s_out.wait_event(done)
+            with torch.cuda.stream(s_out):
+                out_host[:, h0:h1].copy_(sub.out, non_blocking=True)
+        for s in (s_in, s_cmp, s_out):
+            main.wait_stream(s)
+        return out_host
+
     def kernel_launches(self, method: int) -> int:
         """Kernels one forward() launches: drift: pool, scores, drift prep, drift, select,
         schedule, attention; mass / random: pool, fused scores + select, schedule,

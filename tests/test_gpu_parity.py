@@ -317,6 +317,29 @@ def test_schedule_many_rows_and_repeated_counts():
     assert order.cpu().tolist() == sorted(range(384), key=lambda it: (-flat[it], it))
 
 
+@pytest.mark.parametrize("method", ["mass", "drift"])
+def test_host_buffer_path_in_head_groups_equals_forward(method):
+    """forward_host (pinned host tensors, heads in groups on overlapping streams) gives the
+    same bytes as forward() on device tensors: every step is per head."""
+    ensure_built()
+    wl = W.make_workload(2, heads=4, views=6, method=method, sparsity=0.75, rounds=3)
+    dev = torch.device("cuda")
+    B, H, N, _ = wl.q.shape
+    ref = SparseGlobalAttention(B, H, N, device=dev)
+    ref.load_output_projection(wl.w_o.to(dev))
+    ref.forward(wl.q.to(dev), wl.k.to(dev), wl.v.to(dev), METHODS[method], wl.budgets,
+                wl.keep_k.to(dev), wl.dense_q.to(dev), wl.rounds, wl.rho, wl.eps, wl.select_seed)
+    layer = SparseGlobalAttention(B, H, N, device=dev)
+    layer.make_groups(wl.w_o.to(dev), 3)
+    qh, kh, vh = (t.cpu().pin_memory() for t in (wl.q, wl.k, wl.v))
+    outh = torch.empty(B, H, N, 64, dtype=torch.bfloat16).pin_memory()
+    for _ in range(2):
+        layer.forward_host(qh, kh, vh, outh, METHODS[method], wl.budgets, wl.keep_k.to(dev),
+                           wl.dense_q.to(dev), wl.rounds, wl.rho, wl.eps, wl.select_seed)
+    torch.cuda.synchronize()
+    assert torch.equal(outh, ref.out.cpu())
+
+
 def test_wide_logit_range_and_rescaling():
     """Logits spread over hundreds of units (Q scaled by 12): exp2 arguments reach the
     clamp at -126, the running max jumps between tiles and forces O rescales; a ragged
