@@ -34,6 +34,11 @@ Readings of points the pages leave open (each is also listed in the design doc):
                     c candidates with the SMALLEST rank key kappa in the initial selection.
     realized drift  J of a returned selection = Eq. 12 on its drop set (Eq. 10), for any
                     method ([ReSS] §6.1, Figs. 7 and 9); 0 for a dense query block.
+    CDF threshold   SparseVGGT's top-p rule ([ReSS] §2 related work, §4.4, Table 2
+                    "+CDF threshold", Supp. F): candidates in (P descending, block index
+                    ascending) order are kept until the kept mass, always-kept blocks
+                    included, reaches top_p (partial sums in float64), never more than the
+                    budget c and never fewer than one candidate when c >= 1.
 Parity status: every function below is pinned by tests/test_oracle_*.py.  The exact
 swap trajectory of the restoration is pinned only through the readings above and the
 brute-force bounds (J_opt <= J_ress <= J_init); the pages print no trajectory.
@@ -45,7 +50,7 @@ from typing import Optional, Sequence
 
 import numpy as np
 
-MASS, DRIFT, RANDOM = 0, 1, 2
+MASS, DRIFT, RANDOM, CDF = 0, 1, 2, 3
 MINIMISE, MAXIMISE_SWAPS, MAXIMISE_FULL = 0, 1, 2   # drift objective ([ReSS] Fig. 8)
 MASK64 = (1 << 64) - 1
 SPLITMIX_GAMMA = 0x9E3779B97F4A7C15
@@ -233,10 +238,37 @@ def realized_drift(selected: Sequence[int], cand: Sequence[int], P_row, v_pool_h
     return float(objective(g, K, M, eps, dtype)[0])
 
 
+def cdf_keep(P_row, cand: Sequence[int], budget: int, top_p: float, fixed_mass: float):
+    """Top-p selection (reading above): the kept candidates and the smallest relative gap
+    of the decisions (the cumulative mass against top_p where the count was cut, and the
+    probability gap at the cut)."""
+    order = sorted(cand, key=lambda j: (-float(P_row[j]), j))
+    c = max(0, min(budget, len(order)))
+    if c == 0:
+        return [], math.inf
+    cum = float(fixed_mass)
+    n = c
+    sums = []
+    for q, j in enumerate(order[:c]):
+        cum += float(P_row[j])      # python floats: float64
+        sums.append(cum)
+        if cum >= top_p:
+            n = q + 1
+            break
+    n = max(1, n)
+    margin = math.inf
+    if n < c:    # cut by the threshold: how close the sums before and at the cut came
+        before = float(fixed_mass) if n == 1 else sums[n - 2]
+        margin = min(abs(sums[n - 1] - top_p), abs(before - top_p)) / max(top_p, 1e-30)
+    if n < len(order):   # the order itself at the cut
+        margin = min(margin, _rel_gap(float(P_row[order[n - 1]]), float(P_row[order[n]])))
+    return order[:n], margin
+
+
 def select_row(method: int, P_row, cand: Sequence[int], budget: int, *, s_row=None,
                v_pool_head=None, vbar_row=None, M=None, rounds: int = 0, rho: float = 0.5,
-               eps: float = 1e-4, rand_keys=None, sign: int = MINIMISE,
-               dtype=np.float32) -> dict:
+               eps: float = 1e-4, rand_keys=None, sign: int = MINIMISE, top_p: float = 1.0,
+               fixed_mass: float = 0.0, dtype=np.float32) -> dict:
     """Block selection for one (query block, head) row.
 
     `sign` selects the drift objective (drift only): MINIMISE ([ReSS] §4), or the
@@ -267,6 +299,9 @@ def select_row(method: int, P_row, cand: Sequence[int], budget: int, *, s_row=No
     if method == RANDOM:
         sel, _ = top_by_score(cand, {j: rand_keys[j] for j in cand}, c)
         return finish(sel, math.inf)
+    if method == CDF:
+        sel, mg = cdf_keep(P_row, cand, c, top_p, fixed_mass)
+        return finish(sel, mg)
     assert method == DRIFT
     maximise = sign != MINIMISE
     P_row = np.asarray(P_row, dtype=dtype)
@@ -314,7 +349,7 @@ def select_row(method: int, P_row, cand: Sequence[int], budget: int, *, s_row=No
 def select_blocks(method: int, P, budgets: Sequence[int], keep_k=None, dense_q=None, *,
                   s=None, v_pool=None, vbar=None, gram=None, rounds: int = 0, rho: float = 0.5,
                   eps: float = 1e-4, seed: int = 0, rows=None, sign: int = MINIMISE,
-                  dtype=np.float32) -> dict:
+                  top_p: float = 1.0, dtype=np.float32) -> dict:
     """Selection for every (b, h, i) row, or for the listed `rows` only.
 
     Returns dict(kept = {(b,h,i): ascending list of kept key blocks}, margin = {...},
@@ -342,7 +377,8 @@ def select_blocks(method: int, P, budgets: Sequence[int], keep_k=None, dense_q=N
                          v_pool_head=None if v_pool is None else v_pool[b, h],
                          vbar_row=None if vbar is None else vbar[b, h, i],
                          M=None if gram is None else gram[h], rounds=rounds, rho=rho, eps=eps,
-                         rand_keys=rk, sign=sign, dtype=dtype)
+                         rand_keys=rk, sign=sign, top_p=top_p,
+                         fixed_mass=sum(float(P[b, h, i, j]) for j in always), dtype=dtype)
         kept[(b, h, i)] = sorted(always + res["selected"])
         margins[(b, h, i)] = res["margin"]
         info[(b, h, i)] = res

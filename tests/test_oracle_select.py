@@ -251,3 +251,53 @@ def test_realized_drift_of_mass_and_dense_rows():
     assert res["info"][(0, 0, 0)]["J"] == pytest.approx(
         _J_masked(logits, Vp, vbar, W, set(range(8)) - set(kept0)), rel=1e-9)
     assert res["info"][(0, 0, 1)]["J"] == 0.0
+
+
+# ------------------------------------------- CDF / top-p threshold (SparseVGGT's rule)
+def test_cdf_keeps_the_shortest_prefix_reaching_the_threshold():
+    """Against a numpy cumulative sum over the descending order: the smallest n whose
+    mass (always-kept blocks included) reaches top_p, capped by the budget."""
+    rng = np.random.default_rng(11)
+    for trial in range(30):
+        nk = int(rng.integers(4, 40))
+        logits = rng.normal(size=nk) * rng.uniform(0.5, 4)
+        P = np.exp(logits - logits.max())
+        P /= P.sum()
+        fixed = [j for j in range(nk) if rng.random() < 0.1]
+        cand = [j for j in range(nk) if j not in fixed]
+        if not cand:
+            continue
+        c = int(rng.integers(1, len(cand) + 1))
+        tau = float(rng.uniform(0.05, 1.0))
+        order = np.array(cand)[np.argsort(-P[cand], kind="stable")]
+        csum = float(P[fixed].sum()) + np.cumsum(P[order].astype(np.float64))
+        hit = np.nonzero(csum >= tau)[0]
+        n = min(c, max(1, int(hit[0]) + 1 if len(hit) else c))
+        kept, _ = O.cdf_keep(P, cand, c, tau, float(P[fixed].sum()))
+        assert sorted(kept) == sorted(order[:n].tolist()), trial
+
+
+def test_cdf_special_cases():
+    P = np.array([0.5, 0.25, 0.125, 0.0625, 0.0625])
+    cand = list(range(5))
+    assert O.cdf_keep(P, cand, 5, 0.8, 0.0)[0] == [0, 1, 2]        # 0.75 < 0.8 <= 0.875
+    assert O.cdf_keep(P, cand, 2, 0.8, 0.0)[0] == [0, 1]           # capped by the budget
+    assert O.cdf_keep(P, cand, 5, 1e-9, 0.0)[0] == [0]             # at least one candidate
+    assert O.cdf_keep(P, cand[1:], 4, 0.3, 0.5)[0] == [1]          # always-kept mass counts
+    assert O.cdf_keep(P, cand, 0, 0.5, 0.0)[0] == []
+    # top_p = 1 keeps the budget's top-c: the attention-mass selection
+    rng = np.random.default_rng(2)
+    P = rng.dirichlet(np.ones(20))
+    mass = O.select_row(O.MASS, P, list(range(20)), 7)["selected"]
+    cdf = O.select_row(O.CDF, P, list(range(20)), 7, top_p=1.0)["selected"]
+    assert mass == cdf
+
+
+def test_cdf_kept_sets_grow_with_the_threshold():
+    rng = np.random.default_rng(4)
+    P = rng.dirichlet(np.ones(30) * 0.3)
+    prev = set()
+    for tau in np.linspace(0.05, 1.0, 20):
+        kept = set(O.cdf_keep(P, list(range(30)), 30, float(tau), 0.0)[0])
+        assert prev <= kept
+        prev = kept
