@@ -46,7 +46,9 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--case", type=int, default=2, help="synthetic case index (2 = 8 views, mass 50%%)")
-    ap.add_argument("--method", choices=["mass", "drift", "random"], default=None)
+    ap.add_argument("--method", choices=["mass", "drift", "random", "cdf"], default=None)
+    ap.add_argument("--top-p", type=float, default=0.9,
+                    help="mass threshold of the cdf method (the budget from --sparsity caps it)")
     ap.add_argument("--sparsity", type=float, default=None)
     ap.add_argument("--objective", choices=["min", "max-swaps", "max-full"], default="min",
                     help="drift objective: the method, or a drift-maximising control (drift only)")
@@ -212,7 +214,8 @@ def run_ours(args):
     def step():
         if fused:
             layer.pool(q, k, v)
-            layer.scores_select(wl.method, wl.budgets, keep_k, dense_q, wl.select_seed)
+            layer.scores_select(wl.method, wl.budgets, keep_k, dense_q, wl.select_seed,
+                                top_p=args.top_p)
         else:
             layer.scores(q, k, v)
             layer.drift()
@@ -238,7 +241,7 @@ def run_ours(args):
     J = torch.zeros(Bsz, H, layer.nb, device=dev)
     layer.scores(q, k, v)
     layer.select(wl.method, wl.budgets, keep_k, dense_q, wl.rounds, wl.rho, wl.eps, wl.select_seed,
-                 objective=objective, drift_out=J)
+                 objective=objective, drift_out=J, top_p=args.top_p)
     torch.cuda.synchronize()
     sparse_rows = J[:, :, ~wl.dense_q.bool().to(dev)] if wl.dense_q is not None else J
     drift_mean = float(sparse_rows.mean().item())
@@ -273,7 +276,7 @@ def run_ours(args):
                  ["pool", "block_scores", "drift", "select", "schedule", "attention"])
         calls = {
             "scores_select": lambda: layer.scores_select(wl.method, wl.budgets, keep_k, dense_q,
-                                                         wl.select_seed),
+                                                         wl.select_seed, top_p=args.top_p),
             "pool": lambda: R.ress_pool_blocks(layer.shape, q, k, v, layer.q_pool, layer.k_pool, layer.v_pool),
             "block_scores": lambda: R.ress_block_scores(layer.shape, layer.q_pool, layer.k_pool, layer.v_pool,
                                                         layer.scale, layer.P, layer.v_bar),
@@ -330,7 +333,7 @@ def run_ours(args):
                 a.record(stream)
                 layer.forward_host(qh, kh, vh, outh, wl.method, wl.budgets, keep_k, dense_q,
                                    wl.rounds, wl.rho, wl.eps, wl.select_seed, q_dev=qd, k_dev=kd,
-                                   v_dev=vd)
+                                   v_dev=vd, top_p=args.top_p)
                 b.record(stream)
                 torch.cuda.synchronize()
                 if s >= 2:
@@ -358,9 +361,10 @@ def run_ours(args):
         "data": "synthetic (seeded, VGGT-shaped)",
         "config": {
             "workload": wl.case.name, "batch": Bsz, "heads": H, "seq_len": N, "head_dim": 64,
-            "block": 128, "method": ["mass", "drift", "random"][wl.method], "sparsity": wl.sparsity,
+            "block": 128, "method": ["mass", "drift", "random", "cdf"][wl.method], "sparsity": wl.sparsity,
             "rounds": wl.rounds, "budgets": sorted(set(wl.budgets)) if len(set(wl.budgets)) < 4 else "dirichlet",
             "drift_objective": args.objective, "realized_drift_J_mean": float(f"{drift_mean:.6g}"),
+            **({"top_p": args.top_p} if wl.method == R.SELECT_CDF else {}),
             "kept_tile_fraction": round(kept_frac, 4), "kept_tile_gflop": round(flops / 1e9, 3),
             "selection_dtype": "f32", "l2": "flushed before every timed step (256 MiB write)",
             "parallelism": f"{world} independent layers, one per GPU" if world > 1 else "single GPU",
@@ -378,7 +382,7 @@ def run_ours(args):
     if "e2e" in extra:
         line["e2e"] = extra["e2e"]
     if rank == 0 and not args.no_cpu_baseline and world == 1 and not args.quick:
-        line["cpu_baseline"] = cpu_baseline(wl, seconds=15.0)
+        line["cpu_baseline"] = cpu_baseline(wl, seconds=15.0, top_p=args.top_p)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -387,7 +391,7 @@ def run_ours(args):
 
 
 # ------------------------------------------------------------- CPU oracle timing
-def _oracle_sample(wl, heads):
+def _oracle_sample(wl, heads, top_p: float = 1.0):
     """Runs the oracle's whole path for the listed heads of the layer; returns
     (seconds, kept-tile FLOPs of the sample)."""
     import numpy as np
@@ -401,7 +405,7 @@ def _oracle_sample(wl, heads):
     budgets = [wl.budgets[h] for h in heads]
     t0 = time.perf_counter()
     res = O.layer(q, k, v, w_o, wl.method, budgets, wl.keep_k.cpu().numpy(), wl.dense_q.cpu().numpy(),
-                  rounds=wl.rounds, rho=wl.rho, eps=wl.eps, seed=wl.select_seed)
+                  rounds=wl.rounds, rho=wl.rho, eps=wl.eps, seed=wl.select_seed, top_p=top_p)
     dt = time.perf_counter() - t0
     N = q.shape[2]
     valid = [min(128, N - 128 * j) for j in range((N + 127) // 128)]
@@ -418,11 +422,11 @@ def _cores():
         return os.cpu_count() or 1
 
 
-def cpu_baseline(wl, seconds: float = 15.0):
+def cpu_baseline(wl, seconds: float = 15.0, top_p: float = 1.0):
     H = wl.q.shape[1]
     done, tot_t, tot_f, h = [], 0.0, 0.0, 0
     while tot_t < seconds and h < H:
-        dt, fl = _oracle_sample(wl, [h])
+        dt, fl = _oracle_sample(wl, [h], top_p)
         tot_t += dt
         tot_f += fl
         done.append(h)
@@ -445,7 +449,7 @@ def run_reference(args):
     H = wl.q.shape[1]
     times, flops = [], []
     for s in range(args.warmup + args.steps):
-        dt, fl = _oracle_sample(wl, [s % H])
+        dt, fl = _oracle_sample(wl, [s % H], args.top_p)
         if s >= args.warmup:
             times.append(dt)
             flops.append(fl)
@@ -456,7 +460,7 @@ def run_reference(args):
         "ms_per_step": round(1e3 * statistics.mean(times), 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded, VGGT-shaped)",
         "config": {"workload": wl.case.name, "batch": 1, "heads": H, "seq_len": wl.q.shape[2],
-                   "head_dim": 64, "block": 128, "method": ["mass", "drift", "random"][wl.method],
+                   "head_dim": 64, "block": 128, "method": ["mass", "drift", "random", "cdf"][wl.method],
                    "sparsity": wl.sparsity, "rounds": wl.rounds,
                    "step": "oracle whole path for one head of the layer (heads rotate)"},
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",

@@ -136,6 +136,7 @@ __global__ void __launch_bounds__(kPoolWarps * 32) pool_kernel(const uint4 *__re
 // drift method keeps its separate kernels).  P and vbar are then optional outputs.
 struct FusedSelect {
   int method, H;
+  float top_p;
   uint64_t seed;
   const uint8_t *keep_k, *dense_q;
   int32_t *kv_idx, *kv_cnt;
@@ -144,9 +145,10 @@ struct FusedSelect {
 };
 constexpr uint8_t kCand = 0, kFixed = 1, kKept = 2;  // per-block state during selection
 
-// per-warp selection scratch: histogram, gather slots, block states
-__host__ __device__ __forceinline__ size_t fused_warp_bytes(int nb) {
-  return 1024 + 128 + (size_t)((nb + 15) & ~15);
+// per-warp selection scratch: histogram, gather slots, block states, and for the CDF
+// method the kept probabilities in rank order
+__host__ __device__ __forceinline__ size_t fused_warp_bytes(int nb, bool cdf) {
+  return 1024 + 128 + (size_t)((nb + 15) & ~15) + (cdf ? (size_t)((nb + 3) & ~3) * 4 : 0);
 }
 
 template <int TQ, bool SEL>
@@ -214,11 +216,13 @@ __global__ void __launch_bounds__(kThreads) block_scores_kernel(
     // ------------------------------------------------ fused mass / random selection
     // the same decisions as the selection kernel: top-c of the candidates by P (or by
     // the SplitMix64 key), ties to the lower block index; dense rows keep every block
+    const bool cdf = fs.method == RESS_SELECT_CDF;
     unsigned char *wb = reinterpret_cast<unsigned char *>(sl + (size_t)TQ * nb) +
-                        fused_warp_bytes(nb) * warp;
+                        fused_warp_bytes(nb, cdf) * warp;
     uint32_t *hist = reinterpret_cast<uint32_t *>(wb);
     int *slot = reinterpret_cast<int *>(wb + 1024);
     uint8_t *st = wb + 1152;
+    float *sorted = reinterpret_cast<float *>(st + ((nb + 15) & ~15));
     const int h = (int)(bh % fs.H);
 #pragma unroll 1
     for (int q = 0; q < R; ++q) {
@@ -238,8 +242,17 @@ __global__ void __launch_bounds__(kThreads) block_scores_kernel(
       if (!dense) {
         auto is_cand = [&](int j) { return st[j] == kCand; };
         auto keep = [&](int j) { st[j] = kKept; };
-        if (fs.method == RESS_SELECT_MASS) {
+        if (fs.method == RESS_SELECT_MASS || cdf) {
           warp_select<uint32_t>(nb, c, [&](int j) { return float_key(row[j]); }, is_cand, keep, hist, slot);
+          if (cdf) {
+            double fixed = 0.0;  // mass of the always-kept blocks
+            for (int j = lane; j < nb; j += 32)
+              if (st[j] == kFixed) fixed += (double)row[j];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) fixed += __shfl_xor_sync(0xffffffffu, fixed, o);
+            warp_cdf_cut(nb, row, [&](int j) { return st[j] == kKept; }, [&](int j) { st[j] = kCand; },
+                         fixed, fs.top_p, sorted);
+          }
         } else {
           const uint64_t base = ((uint64_t)bh * nb + (uint64_t)i) * (uint64_t)nb;
           warp_select<uint64_t>(nb, c, [&](int j) { return splitmix64_key(fs.seed, base + (uint64_t)j + 1); },
@@ -401,7 +414,7 @@ static cudaError_t scores_tq(const Dims &d, const float *qp, const float *kp, co
                              float scale, float *P, float *vbar, const FusedSelect &fs,
                              cudaStream_t st) {
   const size_t smem = sizeof(float) * (2 * kTileFloats + TQ * kHeadDim + (size_t)TQ * d.nb) +
-                      (SEL ? fused_warp_bytes(d.nb) * kWarps : 0);
+                      (SEL ? fused_warp_bytes(d.nb, fs.method == RESS_SELECT_CDF) * kWarps : 0);
   cudaError_t e = cudaFuncSetAttribute(block_scores_kernel<TQ, SEL>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -431,6 +444,7 @@ cudaError_t launch_block_scores(const Dims &d, const float *qp, const float *kp,
 cudaError_t launch_scores_select(const Dims &d, const ScoresSelectLaunch &a, cudaStream_t st) {
   FusedSelect fs{};
   fs.method = a.method;
+  fs.top_p = a.top_p;
   fs.H = d.H;
   fs.seed = a.seed;
   fs.keep_k = a.keep_k;

@@ -27,6 +27,7 @@ constexpr uint8_t F_CAND = 5;     // candidate before the initial selection
 struct SelectParams {
   int H, nb, method, rounds;
   int objective;  // ress_drift_objective
+  float top_p;    // RESS_SELECT_CDF threshold
   float *drift;   // realized J per row, or null
   float rho, eps;
   uint64_t seed;
@@ -134,8 +135,10 @@ RESS_DEV float objective(float G, float K, float eps) {
 // The stride is 16 bytes past a multiple of 128: every warp's block starts 16-byte
 // aligned (float4 reads of M g), and in the cooperative gain pass, where the lanes of
 // one 8-lane phase read M g of eight different rows, those reads fall on distinct banks.
-__host__ __device__ __forceinline__ size_t select_warp_bytes(int nb) {
-  const size_t b = 1024 + 128 + 256 + 32 + (size_t)nb * 4 + 2 * (size_t)((nb + 15) & ~15);
+// The CDF method appends nb floats (the kept probabilities in rank order).
+__host__ __device__ __forceinline__ size_t select_warp_bytes(int nb, bool cdf = false) {
+  const size_t b = 1024 + 128 + 256 + 32 + (size_t)nb * 4 + 2 * (size_t)((nb + 15) & ~15) +
+                   (cdf ? (size_t)nb * 4 : 0);
   return ((b + 127) & ~(size_t)127) + 16;
 }
 
@@ -158,7 +161,9 @@ __global__ void __launch_bounds__(512) select_kernel(const __grid_constant__ Sel
   float *tiles = reinterpret_cast<float *>(smem_raw);
   float(*sM)[kPad] = reinterpret_cast<float(*)[kPad]>(smem_raw + tile_bytes);
   unsigned char *wbase = smem_raw + tile_bytes + (state ? 64 * kPad * 4 : 0);
-  unsigned char *mine = wbase + select_warp_bytes(nb) * warp;
+  const bool cdf = p.method == RESS_SELECT_CDF;
+  const size_t wbytes = select_warp_bytes(nb, cdf);
+  unsigned char *mine = wbase + wbytes * warp;
   uint32_t *hist = reinterpret_cast<uint32_t *>(mine);
   int *slot = reinterpret_cast<int *>(mine + 1024);
   float *sh = reinterpret_cast<float *>(mine + 1152);
@@ -167,6 +172,7 @@ __global__ void __launch_bounds__(512) select_kernel(const __grid_constant__ Sel
   int *list = reinterpret_cast<int *>(gain);  // block lists reuse the gain array
   uint8_t *flags = mine + 1440 + (size_t)nb * 4;
   uint8_t *best = flags + ((nb + 15) & ~15);
+  float *sorted = reinterpret_cast<float *>(best + ((nb + 15) & ~15));  // CDF only
 
   const long long bh = blockIdx.y;
   const int h = (int)(bh % p.H);
@@ -196,10 +202,19 @@ __global__ void __launch_bounds__(512) select_kernel(const __grid_constant__ Sel
   if (active) {
     auto is_cand = [&](int j) { return flags[j] == F_CAND; };
     auto keep = [&](int j) { flags[j] = F_KEPT; };
-    if (p.method == RESS_SELECT_MASS) {
+    if (p.method == RESS_SELECT_MASS || cdf) {
       for (int j = lane; j < nb; j += 32) gain[j] = prow[j];
       __syncwarp();
       warp_select<uint32_t>(nb, c, [&](int j) { return float_key(gain[j]); }, is_cand, keep, hist, slot);
+      if (cdf) {
+        double fixed = 0.0;  // mass of the always-kept blocks
+        for (int j = lane; j < nb; j += 32)
+          if (flags[j] == F_FIXED) fixed += (double)gain[j];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) fixed += __shfl_xor_sync(0xffffffffu, fixed, o);
+        warp_cdf_cut(nb, gain, [&](int j) { return flags[j] == F_KEPT; },
+                     [&](int j) { flags[j] = F_CAND; }, fixed, p.top_p, sorted);
+      }
     } else if (p.method == RESS_SELECT_RANDOM) {
       const uint64_t base = ((uint64_t)bh * nb + (uint64_t)i) * (uint64_t)nb;
       warp_select<uint64_t>(nb, c, [&](int j) { return splitmix64_key(p.seed, base + (uint64_t)j + 1); },
@@ -307,7 +322,7 @@ __global__ void __launch_bounds__(512) select_kernel(const __grid_constant__ Sel
       {
         const int rr = lane & 15, kp = lane >> 4;
         const bool rlive = rr < T;
-        unsigned char *rb = wbase + select_warp_bytes(nb) * (rlive ? rr : 0);
+        unsigned char *rb = wbase + wbytes * (rlive ? rr : 0);
         const float *rh = reinterpret_cast<const float *>(rb + 1152);
         const float *rs = reinterpret_cast<const float *>(rb + 1408);
         float *rgain = reinterpret_cast<float *>(rb + 1440);
@@ -541,9 +556,9 @@ __global__ void __launch_bounds__(1024) schedule_kernel_par(const int32_t *__res
 
 }  // namespace
 
-static size_t select_smem(int nb, int T, bool restore, bool state) {
+static size_t select_smem(int nb, int T, bool restore, bool state, bool cdf) {
   return (restore ? (size_t)kSelStages * kTileFloats * 4 : 0) + (state ? 64 * kPad * 4 : 0) +
-         select_warp_bytes(nb) * T;
+         select_warp_bytes(nb, cdf) * T;
 }
 
 cudaError_t launch_select(const Dims &d, const SelectLaunch &a, cudaStream_t st) {
@@ -556,6 +571,7 @@ cudaError_t launch_select(const Dims &d, const SelectLaunch &a, cudaStream_t st)
   p.eps = a.eps;
   p.seed = a.seed;
   p.objective = a.objective;
+  p.top_p = a.top_p;
   p.drift = a.drift;
   p.keep_k = a.keep_k;
   p.dense_q = a.dense_q;
@@ -575,9 +591,10 @@ cudaError_t launch_select(const Dims &d, const SelectLaunch &a, cudaStream_t st)
   // maps 16 rows to lanes); without rounds the rows are independent, and 4 per CTA give
   // a grid that fills the GPU at small nb
   int T = restore ? 16 : 4;
-  while (T > 4 && select_smem(d.nb, T, restore, state) > 220 * 1024) T >>= 1;
+  const bool cdf = a.method == RESS_SELECT_CDF;
+  while (T > 4 && select_smem(d.nb, T, restore, state, cdf) > 220 * 1024) T >>= 1;
   p.rows_per_cta = T;
-  const size_t smem = select_smem(d.nb, T, restore, state);
+  const size_t smem = select_smem(d.nb, T, restore, state, cdf);
   cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;

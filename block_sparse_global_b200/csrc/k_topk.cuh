@@ -190,4 +190,66 @@ RESS_DEV void warp_select(int n, int k, KeyFn key, ValidFn valid, MarkFn mark, u
 
 // Eq. 17 swap count: max(1, round-half-up(rho c 2^-(r+1))), capped at |D| and c.
 
+// CDF / top-p cut after a top-c by probability (SparseVGGT's rule): of the kept entries,
+// in (pv descending, index ascending) order, keep the shortest prefix whose sum plus
+// fixed_mass reaches top_p (float64 partial sums), at least one.  pv[j] is entry j's
+// probability, kept(j) / unkeep(j) read and clear its kept state, sorted is warp scratch
+// for at least as many floats as entries are kept.  Warp-collective.
+template <typename KeptFn, typename UnkeepFn>
+RESS_DEV void warp_cdf_cut(int n, const float *pv, KeptFn kept, UnkeepFn unkeep, double fixed_mass,
+                           float top_p, float *sorted) {
+  const int lane = threadIdx.x & 31;
+  auto rank_of = [&](int j) {
+    const float x = pv[j];
+    int r = 0;
+    for (int k = 0; k < n; ++k)
+      if (kept(k)) {
+        const float y = pv[k];
+        r += (y > x || (y == x && k < j)) ? 1 : 0;
+      }
+    return r;
+  };
+  int c = 0;
+  for (int j = lane; j < n; j += 32)
+    if (kept(j)) {
+      sorted[rank_of(j)] = pv[j];
+      ++c;
+    }
+  c = warp_sum_i(c);
+  __syncwarp();
+  // first position whose running sum (plus the always-kept mass) reaches top_p
+  int cut = c;
+  double run = fixed_mass;
+  for (int base = 0; base < c; base += 32) {
+    const int q = base + lane;
+    double incl = q < c ? (double)sorted[q] : 0.0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const double y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const unsigned hit = __ballot_sync(0xffffffffu, q < c && run + incl >= (double)top_p);
+    if (hit) {
+      cut = base + __ffs(hit);
+      break;
+    }
+    run += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  cut = max(1, cut);
+  // decide every drop against the unchanged kept set, then apply (n <= 4096: at most
+  // 128 entries per lane).  Entries above the value at the cut stay, entries below it
+  // go; only entries equal to it need their rank.
+  const float vcut = sorted[cut - 1];
+  uint32_t drop[4] = {0u, 0u, 0u, 0u};
+  for (int j = lane, t = 0; j < n; j += 32, ++t)
+    if (kept(j)) {
+      const float x = pv[j];
+      if (x < vcut || (x == vcut && rank_of(j) >= cut)) drop[t >> 5] |= 1u << (t & 31);
+    }
+  __syncwarp();
+  for (int j = lane, t = 0; j < n; j += 32, ++t)
+    if (drop[t >> 5] & (1u << (t & 31))) unkeep(j);
+  __syncwarp();
+}
+
 }  // namespace ress

@@ -12,7 +12,7 @@ using ress::Dims;
 
 namespace {
 
-constexpr int32_t kAbiVersion = 2;
+constexpr int32_t kAbiVersion = 3;
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -129,8 +129,10 @@ ress_status ress_select_blocks(const ress_shape *shape, const ress_select_params
   if (st != RESS_OK) return st;
   if (params == nullptr || params->budgets == nullptr) return RESS_ERR_INVALID_ARG;
   const int m = params->method;
-  if (m != RESS_SELECT_MASS && m != RESS_SELECT_DRIFT && m != RESS_SELECT_RANDOM)
+  if (m != RESS_SELECT_MASS && m != RESS_SELECT_DRIFT && m != RESS_SELECT_RANDOM &&
+      m != RESS_SELECT_CDF)
     return RESS_ERR_INVALID_ARG;
+  if (m == RESS_SELECT_CDF && !(params->top_p > 0.f && params->top_p <= 1.f)) return RESS_ERR_INVALID_ARG;
   for (int h = 0; h < d.H; ++h)
     if (params->budgets[h] < 0 || params->budgets[h] > d.nb) return RESS_ERR_INVALID_ARG;
   const int obj = params->objective;
@@ -158,6 +160,7 @@ ress_status ress_select_blocks(const ress_shape *shape, const ress_select_params
   a.rho = params->rho;
   a.eps = (m == RESS_SELECT_DRIFT || want_drift) ? params->eps : 1e-4f;
   a.objective = obj;
+  a.top_p = params->top_p;
   a.drift = params->drift;
   a.seed = params->seed;
   a.budgets = params->budgets;
@@ -187,7 +190,8 @@ ress_status ress_scores_select(const ress_shape *shape, const ress_select_params
   if (params == nullptr || params->budgets == nullptr) return RESS_ERR_INVALID_ARG;
   const int m = params->method;
   if (m == RESS_SELECT_DRIFT) return RESS_ERR_UNSUPPORTED;
-  if (m != RESS_SELECT_MASS && m != RESS_SELECT_RANDOM) return RESS_ERR_INVALID_ARG;
+  if (m != RESS_SELECT_MASS && m != RESS_SELECT_RANDOM && m != RESS_SELECT_CDF) return RESS_ERR_INVALID_ARG;
+  if (m == RESS_SELECT_CDF && !(params->top_p > 0.f && params->top_p <= 1.f)) return RESS_ERR_INVALID_ARG;
   if (params->objective != RESS_DRIFT_MINIMISE || params->drift != nullptr) return RESS_ERR_INVALID_ARG;
   for (int h = 0; h < d.H; ++h)
     if (params->budgets[h] < 0 || params->budgets[h] > d.nb) return RESS_ERR_INVALID_ARG;
@@ -201,6 +205,7 @@ ress_status ress_scores_select(const ress_shape *shape, const ress_select_params
   ress::ScoresSelectLaunch a;
   a.method = m;
   a.seed = params->seed;
+  a.top_p = params->top_p;
   a.budgets = params->budgets;
   a.keep_k = params->keep_k;
   a.dense_q = params->dense_q;

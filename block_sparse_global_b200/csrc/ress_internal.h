@@ -26,6 +26,7 @@ cudaError_t launch_block_scores(const Dims &d, const float *qp, const float *kp,
 // Block map fused with mass / random selection (P and vbar optional).
 struct ScoresSelectLaunch {
   int method;
+  float top_p;
   uint64_t seed;
   const int32_t *budgets;  // host [H]
   const uint8_t *keep_k, *dense_q;
@@ -43,6 +44,7 @@ cudaError_t launch_drift(const Dims &d, const float *P, const float *vp, const f
 
 struct SelectLaunch {
   int method, rounds, objective;
+  float top_p;    // RESS_SELECT_CDF threshold
   float *drift;  // realized J per row, or null
   float rho, eps;
   uint64_t seed;

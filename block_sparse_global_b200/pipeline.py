@@ -58,10 +58,10 @@ class SparseGlobalAttention:
                             self.v_bar, stream)
 
     def scores_select(self, method: int, budgets: Sequence[int], keep_k=None, dense_q=None,
-                      seed: int = 0, write_scores: bool = False, stream=None):
-        """Block map and MASS / RANDOM selection in one kernel (after pool()).  P and v_bar
-        are written only with write_scores."""
-        params = R.select_params(method, budgets, keep_k, dense_q, 0, 0.5, 1e-4, seed)
+                      seed: int = 0, write_scores: bool = False, stream=None, top_p: float = 1.0):
+        """Block map and MASS / CDF / RANDOM selection in one kernel (after pool()).  P and
+        v_bar are written only with write_scores."""
+        params = R.select_params(method, budgets, keep_k, dense_q, 0, 0.5, 1e-4, seed, top_p=top_p)
         R.ress_scores_select(self.shape, params, self.q_pool, self.k_pool,
                              self.v_pool if write_scores else None, self.scale,
                              self.P if write_scores else None,
@@ -74,12 +74,13 @@ class SparseGlobalAttention:
 
     def select(self, method: int, budgets: Sequence[int], keep_k=None, dense_q=None, rounds: int = 0,
                rho: float = 0.5, eps: float = 1e-4, seed: int = 0, stream=None,
-               objective: int = R.DRIFT_MINIMISE, drift_out: Optional[torch.Tensor] = None):
+               objective: int = R.DRIFT_MINIMISE, drift_out: Optional[torch.Tensor] = None,
+               top_p: float = 1.0):
         """Block selection.  `objective` flips the sign of the drift objective (the
         maximising controls, drift only); `drift_out` (fp32 [B,H,nb]) receives each row's
         realized drift J."""
         params = R.select_params(method, budgets, keep_k, dense_q, rounds, rho, eps, seed,
-                                 objective, drift_out)
+                                 objective, drift_out, top_p)
         drift = method == R.SELECT_DRIFT
         state = drift or drift_out is not None
         R.ress_select_blocks(self.shape, params, self.P, self.s if drift else None,
@@ -95,14 +96,15 @@ class SparseGlobalAttention:
                                  self.dev_err, stream)
 
     def forward(self, q, k, v, method: int, budgets: Sequence[int], keep_k=None, dense_q=None,
-                rounds: int = 0, rho: float = 0.5, eps: float = 1e-4, seed: int = 0, stream=None):
+                rounds: int = 0, rho: float = 0.5, eps: float = 1e-4, seed: int = 0, stream=None,
+                top_p: float = 1.0):
         if method == R.SELECT_DRIFT:
             self.scores(q, k, v, stream)
             self.drift(stream)
             self.select(method, budgets, keep_k, dense_q, rounds, rho, eps, seed, stream)
         else:   # the block map and the selection fused in one kernel
             self.pool(q, k, v, stream)
-            self.scores_select(method, budgets, keep_k, dense_q, seed, stream=stream)
+            self.scores_select(method, budgets, keep_k, dense_q, seed, stream=stream, top_p=top_p)
         self.attend(q, k, v, stream)
         return self.out
 
@@ -125,7 +127,8 @@ class SparseGlobalAttention:
 
     def forward_host(self, q_host, k_host, v_host, out_host, method: int, budgets: Sequence[int],
                      keep_k=None, dense_q=None, rounds: int = 0, rho: float = 0.5,
-                     eps: float = 1e-4, seed: int = 0, q_dev=None, k_dev=None, v_dev=None):
+                     eps: float = 1e-4, seed: int = 0, q_dev=None, k_dev=None, v_dev=None,
+                     top_p: float = 1.0):
         """The layer end to end from pinned host tensors [1,H,N,64] bf16 to the pinned host
         output.  Heads are processed in the groups of make_groups(): the copy in of group
         g+1, the kernels of group g and the copy out of group g-1 run on three streams and
@@ -154,7 +157,7 @@ class SparseGlobalAttention:
             with torch.cuda.stream(s_cmp):
                 sub.forward(q_dev[:, h0:h1], k_dev[:, h0:h1], v_dev[:, h0:h1], method,
                             list(budgets)[h0:h1], keep_k, dense_q, rounds, rho, eps, seed,
-                            stream=s_cmp)
+                            stream=s_cmp, top_p=top_p)
                 done = torch.cuda.Event()
                 done.record(s_cmp)
             s_out.wait_event(done)

@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_PKG, "libress.so")
 RESS_OK = 0
 STATUS_NAMES = {0: "RESS_OK", 1: "RESS_ERR_INVALID_ARG", 2: "RESS_ERR_UNSUPPORTED",
                 3: "RESS_ERR_CUDA", 4: "RESS_ERR_DEVICE_BOUNDS", 5: "RESS_ERR_DEVICE_TIMEOUT"}
-SELECT_MASS, SELECT_DRIFT, SELECT_RANDOM = 0, 1, 2
+SELECT_MASS, SELECT_DRIFT, SELECT_RANDOM, SELECT_CDF = 0, 1, 2, 3
 DRIFT_MINIMISE, DRIFT_MAXIMISE_SWAPS, DRIFT_MAXIMISE_FULL = 0, 1, 2
 HEAD_DIM, BLOCK = 64, 128
 
@@ -40,7 +40,8 @@ class ress_select_params(ctypes.Structure):
     _fields_ = [("method", ctypes.c_int32), ("budgets", ctypes.POINTER(ctypes.c_int32)),
                 ("keep_k", ctypes.c_void_p), ("dense_q", ctypes.c_void_p),
                 ("rounds", ctypes.c_int32), ("rho", ctypes.c_float), ("eps", ctypes.c_float),
-                ("seed", ctypes.c_uint64), ("objective", ctypes.c_int32), ("drift", ctypes.c_void_p)]
+                ("seed", ctypes.c_uint64), ("objective", ctypes.c_int32), ("top_p", ctypes.c_float),
+                ("drift", ctypes.c_void_p)]
 
 
 _lib = None
@@ -166,13 +167,13 @@ def ress_drift_scores_static(shape, P, v_pool, v_bar, gram, s, stream=None):
 
 def select_params(method: int, budgets: Sequence[int], keep_k=None, dense_q=None, rounds: int = 0,
                   rho: float = 0.5, eps: float = 1e-4, seed: int = 0, objective: int = 0,
-                  drift=None):
+                  drift=None, top_p: float = 1.0):
     """Packs ress_select_params (`drift`: optional fp32 [B,H,nb] device tensor for the
     realized J per row).  Returns (struct, host budget array that must stay alive)."""
     arr = (ctypes.c_int32 * len(budgets))(*[int(b) for b in budgets])
     p = ress_select_params(int(method), ctypes.cast(arr, ctypes.POINTER(ctypes.c_int32)),
                            _ptr(keep_k), _ptr(dense_q), int(rounds), float(rho), float(eps),
-                           int(seed) & ((1 << 64) - 1), int(objective), _ptr(drift))
+                           int(seed) & ((1 << 64) - 1), int(objective), float(top_p), _ptr(drift))
     return p, arr
 
 

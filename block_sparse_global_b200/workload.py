@@ -45,7 +45,9 @@ VIEW_TOKENS = VIEW_PATCH + VIEW_SPECIAL
 METHOD_MASS = 0
 METHOD_DRIFT = 1
 METHOD_RANDOM = 2
-METHOD_NAMES = {"mass": METHOD_MASS, "drift": METHOD_DRIFT, "random": METHOD_RANDOM}
+METHOD_CDF = 3
+METHOD_NAMES = {"mass": METHOD_MASS, "drift": METHOD_DRIFT, "random": METHOD_RANDOM,
+                "cdf": METHOD_CDF}
 
 
 @dataclass(frozen=True)

@@ -72,8 +72,12 @@ typedef enum {
   RESS_SELECT_DRIFT = 1,  /* ReSS: top-c_h by s_ij / max(1 - P_ij, eps) (Eq. 7), then
                              `rounds` rounds of budget-neutral swaps (Eqs. 13-17) with
                              track-best ([ReSS] §4.2-4.3)                            */
-  RESS_SELECT_RANDOM = 2  /* c_h candidates chosen at random (the random-selection
+  RESS_SELECT_RANDOM = 2, /* c_h candidates chosen at random (the random-selection
                              control of [ReSS] §6.1, Fig. 8)                         */
+  RESS_SELECT_CDF = 3     /* SparseVGGT's top-p rule ([ReSS] §2, §4.4, Table 2 "+CDF
+                             threshold", Supp. F): candidates by P descending are kept
+                             until the kept mass, always-kept blocks included, reaches
+                             top_p (float64 partial sums); at most c_h, at least one  */
 } ress_method;
 
 /* Sign of the drift objective for RESS_SELECT_DRIFT.  The maximising settings are the
@@ -118,6 +122,8 @@ typedef struct {
                                seeded with `seed` (Steele, Lea, Flood, OOPSLA 2014)   */
   int32_t objective;        /* ress_drift_objective; must be RESS_DRIFT_MINIMISE unless
                                method is RESS_SELECT_DRIFT (else INVALID_ARG)          */
+  float top_p;              /* RESS_SELECT_CDF: mass threshold in (0, 1] (else INVALID_ARG);
+                               ignored by the other methods                         */
   float *drift;             /* DEVICE fp32 [B,H,nb] output or NULL: the realized drift J
                                of every row's final selection, Eq. 12 on its drop set
                                (Eq. 10) with K guarded by eps, for any method ([ReSS]
@@ -125,8 +131,8 @@ typedef struct {
                                v_pool, v_bar and gram, and eps > 0.                 */
 } ress_select_params;
 
-/* Version of this ABI (incremented on any incompatible change): 2 (ress_select_params
- * gained `objective` and `drift`). */
+/* Version of this ABI (incremented on any incompatible change): 3 (ress_select_params
+ * gained `objective`, `top_p` and `drift`; RESS_SELECT_CDF). */
 int32_t ress_abi_version(void);
 
 /* Human-readable name of a status code (static string). */
@@ -220,6 +226,7 @@ ress_status ress_drift_scores_static(const ress_shape *shape, const float *P,
  * keeps every key block.  Any other row keeps the always-kept blocks plus c_h
  * candidates chosen by params->method:
  *   MASS   : largest P_ij;
+ *   CDF    : largest P_ij, cut at the top_p mass (see RESS_SELECT_CDF);
  *   RANDOM : largest SplitMix64 key (see ress_select_params.seed);
  *   DRIFT  : largest s_ij / max(1 - P_ij, eps); then for r = 0..R-1, with the drop set
  *            D and its net drift g = sum_D P_ij (v_bar_i - v_pool_j), K = 1 - sum_D P_ij,
@@ -253,7 +260,7 @@ ress_status ress_select_blocks(const ress_shape *shape, const ress_select_params
  * shared memory from its softmax to its top-c, [ReSS] §4.3 "Fused kernel
  * implementation" on the fusion motive).  The kept lists are identical to those of the
  * two separate calls on the same pooled inputs.
- *   params   as for ress_select_blocks; method must be MASS or RANDOM (else
+ *   params   as for ress_select_blocks; method must be MASS, CDF or RANDOM (else
  *            UNSUPPORTED: drift selection needs the drift score and restoration of
  *            its own calls), objective MINIMISE and drift NULL (else INVALID_ARG).
  *   q_pool, k_pool  fp32 [B,H,nb,64] (ress_pool_blocks); v_pool needed only with v_bar.

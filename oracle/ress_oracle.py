@@ -430,7 +430,7 @@ def to_numpy_f32(t) -> np.ndarray:
 
 def layer(q, k, v, w_o, method: int, budgets, keep_k=None, dense_q=None, rounds: int = 0,
           rho: float = 0.5, eps: float = 1e-4, seed: int = 0, rows=None,
-          attn_rows=None, block: int = 128) -> dict:
+          attn_rows=None, block: int = 128, top_p: float = 1.0) -> dict:
     """The whole path for one layer: pool -> P, vbar -> drift -> select -> attention.
     `rows` limits drift and selection to those (b,h,i); `attn_rows` limits the attention
     (default: the selected rows)."""
@@ -449,7 +449,8 @@ def layer(q, k, v, w_o, method: int, budgets, keep_k=None, dense_q=None, rounds:
         for (b, h, i) in rows:
             s[b, h, i] = drift_row(P[b, h, i], vbar[b, h, i], vp[b, h], gram[h])
     sel = select_blocks(method, P, budgets, keep_k, dense_q, s=s, v_pool=vp, vbar=vbar,
-                        gram=gram, rounds=rounds, rho=rho, eps=eps, seed=seed, rows=rows)
+                        gram=gram, rounds=rounds, rho=rho, eps=eps, seed=seed, rows=rows,
+                        top_p=top_p)
     attn = block_sparse_attn(qf, kf, vf, sel["kept"], scale,
                              rows=rows if attn_rows is None else attn_rows, block=block)
     return dict(q_pool=qp, k_pool=kp, v_pool=vp, P=P, vbar=vbar, gram=gram, s=s,

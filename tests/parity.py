@@ -80,7 +80,7 @@ class OracleLayer:
         return s
 
     def select(self, rows, method, rounds, seed, P=None, s_rows=None, vp=None, vbar=None,
-               sign=O.MINIMISE):
+               sign=O.MINIMISE, top_p=1.0):
         P = self.P if P is None else P
         vp = self.vp if vp is None else vp
         vbar = self.vbar if vbar is None else vbar
@@ -92,7 +92,8 @@ class OracleLayer:
                 s_full[r] = val
         return O.select_blocks(method, P, self.wl.budgets, self.keep_k, self.dense_q, s=s_full,
                                v_pool=vp, vbar=vbar, gram=self.gram, rounds=rounds,
-                               rho=self.wl.rho, eps=self.wl.eps, seed=seed, rows=rows, sign=sign)
+                               rho=self.wl.rho, eps=self.wl.eps, seed=seed, rows=rows, sign=sign,
+                               top_p=top_p)
 
     def attention(self, kept, rows):
         return O.block_sparse_attn(self.q, self.k, self.v, kept, self.scale, rows=rows)

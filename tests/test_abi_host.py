@@ -39,7 +39,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert R.ress_abi_version() == 2
+    assert R.ress_abi_version() == 3
     assert R.ress_status_string(0) == "RESS_OK"
     assert R.ress_status_string(5) == "RESS_ERR_DEVICE_TIMEOUT"
     assert R.ress_status_string(99) == "RESS_ERR_UNKNOWN"
@@ -106,6 +106,9 @@ def test_select_parameter_validation(lib):
     p, keep = R.select_params(1, [4, 4], rounds=2, objective=3)
     assert lib.ress_select_blocks(shape, ctypes.byref(p), *args) == INVALID
     # the realized-drift output needs the pooled values, vbar and M, and a valid eps
+    for bad in (0.0, -0.5, 1.5, float("nan")):   # the CDF threshold lies in (0, 1]
+        p, keep = R.select_params(3, [4, 4], top_p=bad)
+        assert lib.ress_select_blocks(shape, ctypes.byref(p), *args) == INVALID
     p, keep = R.select_params(0, [4, 4])
     p.drift = FAKE   # an aligned address that validation rejects before any use
     assert lib.ress_select_blocks(shape, ctypes.byref(p), FAKE, None, None, None, None, FAKE, FAKE,

@@ -104,6 +104,34 @@ def test_selection_alone_on_oracle_scores():
             assert stats["agreement"] == 1.0
 
 
+@pytest.mark.parametrize("top_p", [0.3, 0.6, 0.85, 0.97])
+def test_cdf_selection_on_oracle_scores(top_p):
+    """SparseVGGT's top-p rule on the oracle's own P: kept lists against the oracle, in
+    the selection kernel and in the fused block-map kernel (bit-identical to each other)."""
+    wl = W.make_workload(2, heads=4, views=6, method="mass", sparsity=0.5)
+    ensure_built()
+    orc = OracleLayer(wl)
+    rows = _all_rows(1, 4, orc.nb)
+    dev = torch.device("cuda")
+    layer = SparseGlobalAttention(1, 4, wl.q.shape[2], device=dev, with_mask=True)
+    layer.P.copy_(torch.from_numpy(orc.P))
+    layer.select(O.CDF, wl.budgets, wl.keep_k.to(dev), wl.dense_q.to(dev), top_p=top_p)
+    torch.cuda.synchronize()
+    sel = orc.select(rows, O.CDF, 0, 0, top_p=top_p)
+    stats = compare_masks(layer.kept_lists(), sel, orc.nb, f"cdf/{top_p}")
+    kept = sum(len(v) for v in layer.kept_lists().values())
+    assert stats["rows"] == len(rows) and kept > len(rows)
+    # the fused kernel on the same workload's own pooled inputs against the separate calls
+    ref = SparseGlobalAttention(1, 4, wl.q.shape[2], device=dev, with_mask=True)
+    ref.scores(wl.q.to(dev), wl.k.to(dev), wl.v.to(dev))
+    ref.select(O.CDF, wl.budgets, wl.keep_k.to(dev), wl.dense_q.to(dev), top_p=top_p)
+    fz = SparseGlobalAttention(1, 4, wl.q.shape[2], device=dev, with_mask=True)
+    fz.pool(wl.q.to(dev), wl.k.to(dev), wl.v.to(dev))
+    fz.scores_select(O.CDF, wl.budgets, wl.keep_k.to(dev), wl.dense_q.to(dev), top_p=top_p)
+    torch.cuda.synchronize()
+    assert torch.equal(fz.kv_cnt, ref.kv_cnt) and torch.equal(fz.mask, ref.mask)
+
+
 @pytest.mark.parametrize("method", [O.MASS, O.RANDOM])
 @pytest.mark.parametrize("case", [1, 2])
 def test_fused_scores_select_equals_separate_calls(case, method):

@@ -67,7 +67,7 @@ def _reference_worker(rank: int, world: int, port: int, out) -> None:
         import bench
 
         class A:
-            case, method, sparsity, steps, warmup = 1, None, None, 1, 0
+            case, method, sparsity, steps, warmup, top_p = 1, None, None, 1, 0, 1.0
         buf = io.StringIO()
         with contextlib.redirect_stdout(buf):
             bench.run_reference(A)
@@ -76,17 +76,27 @@ def _reference_worker(rank: int, world: int, port: int, out) -> None:
         dist.destroy_process_group()
 
 
+def _guarded(worker, rank, world, port, out):
+    """Runs a worker; an exception is sent to the parent instead of leaving it waiting."""
+    try:
+        worker(rank, world, port, out)
+    except BaseException as e:  # noqa: BLE001 - reported to the parent, then re-raised
+        out.put((rank, "error", repr(e)))
+        raise
+
+
 def _run(worker, world: int = 2, timeout: float = 240.0):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=worker, args=(r, world, port, q)) for r in range(world)]
+    procs = [ctx.Process(target=_guarded, args=(worker, r, world, port, q)) for r in range(world)]
     for p in procs:
         p.start()
     res = {}
     try:
         for _ in range(world):
             item = q.get(timeout=timeout)
+            assert not (len(item) == 3 and item[1] == "error"), f"rank {item[0]} failed: {item[2]}"
             res[item[0]] = item[1:]
     finally:
         for p in procs:
