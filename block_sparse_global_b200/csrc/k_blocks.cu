@@ -124,6 +124,30 @@ __global__ void __launch_bounds__(kPoolWarps * 32) pool_kernel(const uint4 *__re
   }
 }
 
+// ----------------------------------- special tokens to the tail, [ReSS] Supp. F sink rule
+// One warp moves four token rows (8 lanes x 16 bytes each) per step, grid-stride over
+// the B*H*N rows.  Row r of a head maps to row perm(r) (forward) or perm^-1(r).
+__global__ void __launch_bounds__(kThreads) token_gather_kernel(const uint4 *__restrict__ src,
+                                                                uint4 *__restrict__ dst,
+                                                                long long rows, int N, int T,
+                                                                int S, int V, int inverse) {
+  const int lane = threadIdx.x & 31, sub = lane >> 3, cg = lane & 7;
+  const int Pv = T - S;
+  const long long warps = (long long)gridDim.x * kWarps;
+  for (long long base = ((long long)blockIdx.x * kWarps + (threadIdx.x >> 5)) * 4; base < rows;
+       base += warps * 4) {
+    const long long r = base + sub;
+    if (r >= rows) continue;
+    const long long head = r / N;
+    const int t = (int)(r - head * N);  // token index within the head, view order
+    const int v = t / T, w = t - v * T;
+    const int tail = w < S ? V * Pv + v * S + w : v * Pv + (w - S);  // its place at the tail layout
+    const long long from = head * N + (inverse ? tail : t);
+    const long long to = head * N + (inverse ? t : tail);
+    dst[to * 8 + cg] = src[from * 8 + cg];
+  }
+}
+
 // ---------------------------------------- pooled block map and Eq. 1 output, [ReSS] §4.1
 // One CTA per (b*h, TQ query blocks); warp w owns rows w*R .. w*R+R-1 (R = TQ/8).  The
 // logits of the CTA's rows against every key block stay in shared memory ([TQ][nb]
@@ -395,6 +419,17 @@ __global__ void __launch_bounds__(kThreads) drift_kernel(
 
 cudaError_t launch_head_gram(int H, int d_model, const float *w_o, float *gram, cudaStream_t st) {
   head_gram_kernel<<<H, kThreads, 0, st>>>(w_o, gram, H, d_model);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_token_gather(const Dims &d, int views, int specials, bool inverse,
+                                const void *src, void *dst, cudaStream_t st) {
+  const long long rows = d.BH() * d.N;
+  long long blocks = (rows + 4 * kWarps - 1) / (4 * kWarps);
+  if (blocks > 148 * 32) blocks = 148 * 32;
+  token_gather_kernel<<<(unsigned)blocks, kThreads, 0, st>>>(
+      static_cast<const uint4 *>(src), static_cast<uint4 *>(dst), rows, d.N, d.N / views, specials,
+      views, inverse ? 1 : 0);
   return cudaGetLastError();
 }
 

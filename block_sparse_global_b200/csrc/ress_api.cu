@@ -66,6 +66,21 @@ ress_status ress_head_gram(const ress_shape *shape, int32_t d_model, const float
   return from_cuda(ress::launch_head_gram(d.H, d_model, w_o, gram, (cudaStream_t)stream));
 }
 
+ress_status ress_token_gather(const ress_shape *shape, int32_t views, int32_t specials,
+                              int32_t inverse, const void *src, void *dst, ress_stream_t stream) {
+  Dims d;
+  bool empty;
+  ress_status st = check_shape(shape, &d, &empty);
+  if (st != RESS_OK) return st;
+  if (views < 1 || (d.N > 0 && d.N % views != 0)) return RESS_ERR_INVALID_ARG;
+  if (specials < 0 || specials > d.N / views) return RESS_ERR_INVALID_ARG;
+  if (inverse != 0 && inverse != 1) return RESS_ERR_INVALID_ARG;
+  if (empty) return RESS_OK;
+  if (!ptr_ok(src) || !ptr_ok(dst) || src == dst) return RESS_ERR_INVALID_ARG;
+  return from_cuda(ress::launch_token_gather(d, views, specials, inverse != 0, src, dst,
+                                             (cudaStream_t)stream));
+}
+
 ress_status ress_pool_blocks(const ress_shape *shape, const void *q, const void *k,
                              const void *v, float *q_pool, float *k_pool, float *v_pool,
                              ress_stream_t stream) {

@@ -17,6 +17,9 @@ struct Dims {
 
 cudaError_t launch_head_gram(int H, int d_model, const float *w_o, float *gram, cudaStream_t st);
 
+cudaError_t launch_token_gather(const Dims &d, int views, int specials, bool inverse,
+                                const void *src, void *dst, cudaStream_t st);
+
 cudaError_t launch_pool(const Dims &d, const void *q, const void *k, const void *v, float *qp,
                         float *kp, float *vp, cudaStream_t st);
 

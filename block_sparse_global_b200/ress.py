@@ -51,6 +51,7 @@ _SIGS = {
     "ress_abi_version": (_I32, []),
     "ress_status_string": (ctypes.c_char_p, [_I32]),
     "ress_head_gram": (_I32, [ctypes.POINTER(ress_shape), _I32, _VP, _VP, _VP]),
+    "ress_token_gather": (_I32, [ctypes.POINTER(ress_shape), _I32, _I32, _I32, _VP, _VP, _VP]),
     "ress_pool_blocks": (_I32, [ctypes.POINTER(ress_shape), _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     "ress_block_scores": (_I32, [ctypes.POINTER(ress_shape), _VP, _VP, _VP, ctypes.c_float, _VP,
                                  _VP, _VP]),
@@ -202,6 +203,13 @@ def ress_scores_select(shape, params, q_pool, k_pool, v_pool, scale: float, P, v
                                    _stream(stream))
     del keep
     _check("ress_scores_select", st)
+
+
+def ress_token_gather(shape, views: int, specials: int, inverse: bool, src, dst, stream=None):
+    """Moves every view's special tokens to the tail (inverse=False) or back."""
+    st = load().ress_token_gather(ctypes.byref(_shape(shape)), int(views), int(specials),
+                                  1 if inverse else 0, _ptr(src), _ptr(dst), _stream(stream))
+    _check("ress_token_gather", st)
 
 
 def ress_attn_schedule(shape, kv_cnt, work_order, stream=None):

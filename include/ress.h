@@ -139,6 +139,26 @@ int32_t ress_abi_version(void);
 const char *ress_status_string(ress_status status);
 
 /*
+ * ress_token_gather -- the token layout of the sink rule ([ReSS] Supp. F: "the sink rule
+ * that always keeps the trailing block holding the special tokens"; §3: special tokens
+ * are excluded from sparsification).  A multi-view sequence holds V views of T = S + Pv
+ * tokens each, every view's S special tokens (VGGT: camera, then registers) first.
+ * Forward (inverse = 0) moves every view's patch tokens, in view order, to the front and
+ * every view's special tokens, in view order, to the tail:
+ *   dst[.., v*Pv + p, :] = src[.., v*T + S + p, :]      (patch p of view v)
+ *   dst[.., V*Pv + v*S + t, :] = src[.., v*T + t, :]    (special token t of view v)
+ * so that the trailing key blocks hold every special token (mark them keep_k, and the
+ * query blocks that hold them dense_q).  inverse = 1 applies the reverse permutation
+ * (to bring the attention output back to the view order).
+ *   src, dst  bf16 [B,H,N,64], N = V*T, distinct buffers (else INVALID_ARG).
+ *   views V >= 1, specials S with 0 <= S <= T (INVALID_ARG otherwise or if V does not
+ *   divide N).  A pure row permutation: bit-exact.
+ */
+ress_status ress_token_gather(const ress_shape *shape, int32_t views, int32_t specials,
+                              int32_t inverse, const void *src, void *dst,
+                              ress_stream_t stream);
+
+/*
  * ress_head_gram -- per-head Gram matrices M_h = (W_O^h)^T W_O^h ([ReSS] §4.2, Eq. 8),
  * computed once per layer ("at model load time").
  *   w_o   fp32 [d_model, H*64] row-major: the layer's output projection; head h is the

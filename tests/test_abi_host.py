@@ -118,6 +118,20 @@ def test_select_parameter_validation(lib):
     assert lib.ress_select_blocks(shape, ctypes.byref(p), *args) == INVALID
 
 
+def test_token_gather_validation(lib):
+    shape = ctypes.byref(R.make_shape(1, 2, 10 * 140))   # 10 views of 140 tokens
+    ok = [FAKE, FAKE + 4096, None]
+    assert lib.ress_token_gather(shape, 0, 5, 0, *ok) == INVALID      # no views
+    assert lib.ress_token_gather(shape, 3, 5, 0, *ok) == INVALID      # 3 does not divide N
+    assert lib.ress_token_gather(shape, 10, 141, 0, *ok) == INVALID   # more specials than tokens
+    assert lib.ress_token_gather(shape, 10, -1, 0, *ok) == INVALID
+    assert lib.ress_token_gather(shape, 10, 5, 2, *ok) == INVALID     # inverse is 0 or 1
+    assert lib.ress_token_gather(shape, 10, 5, 0, FAKE, FAKE, None) == INVALID   # in place
+    assert lib.ress_token_gather(shape, 10, 5, 0, FAKE + 8, FAKE + 4096, None) == INVALID
+    assert lib.ress_token_gather(ctypes.byref(R.make_shape(0, 2, 1400)), 10, 5, 0, None, None,
+                                 None) == OK
+
+
 def test_fused_scores_select_validation(lib):
     shape = ctypes.byref(R.make_shape(1, 2, 1024))
     args = [FAKE, FAKE, FAKE, 0.125, None, None, FAKE, FAKE, None, None, None]

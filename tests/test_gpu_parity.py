@@ -368,6 +368,63 @@ def test_host_buffer_path_in_head_groups_equals_forward(method):
     assert torch.equal(outh, ref.out.cpu())
 
 
+def _tail_order(V, T, S):
+    """Position of every view-order token after the sink-rule permutation (the layout of
+    ress_token_gather written out with numpy)."""
+    t = np.arange(V * T)
+    v, w = t // T, t % T
+    return np.where(w < S, V * (T - S) + v * S + w, v * (T - S) + (w - S))
+
+
+@pytest.mark.parametrize("V,T,S", [(8, 1374, 5), (3, 300, 0), (4, 129, 129), (7, 200, 1)])
+def test_token_gather_matches_the_layout_and_inverts(V, T, S):
+    ensure_built()
+    g = torch.Generator(device="cuda").manual_seed(V * T + S)
+    x = torch.randn(2, 3, V * T, 64, device="cuda", generator=g).to(torch.bfloat16)
+    shape = R.make_shape(2, 3, V * T)
+    y = torch.empty_like(x)
+    R.ress_token_gather(shape, V, S, False, x, y)
+    back = torch.empty_like(x)
+    R.ress_token_gather(shape, V, S, True, y, back)
+    torch.cuda.synchronize()
+    pos = torch.from_numpy(_tail_order(V, T, S)).cuda()
+    want = torch.empty_like(x)
+    want[:, :, pos] = x
+    assert torch.equal(y, want)
+    assert torch.equal(back, x)
+
+
+def test_layer_in_view_order_through_the_sink_rule():
+    """A layer whose tokens come in VGGT's view order (every view's 5 special tokens
+    first): gather to the tail layout, run the layer (the trailing blocks holding the
+    special tokens are always kept), gather the output back.  Equal, bit for bit, to the
+    layer on the tail layout with its output permuted back."""
+    ensure_built()
+    wl = W.make_workload(2, heads=4, views=6, device="cuda")
+    dev = torch.device("cuda")
+    B, H, N, _ = wl.q.shape
+    V, S = 6, 5
+    pos = torch.from_numpy(_tail_order(V, N // V, S)).cuda()
+    ref = SparseGlobalAttention(B, H, N, device=dev)
+    ref.load_output_projection(wl.w_o)
+    ref.forward(wl.q, wl.k, wl.v, wl.method, wl.budgets, wl.keep_k, wl.dense_q, wl.rounds,
+                wl.rho, wl.eps, wl.select_seed)
+    shape = R.make_shape(B, H, N)
+    view_order = [x[:, :, pos] for x in (wl.q, wl.k, wl.v)]   # token t of view order
+    tail = [torch.empty_like(x) for x in view_order]
+    for src, dst in zip(view_order, tail):
+        R.ress_token_gather(shape, V, S, False, src.contiguous(), dst)
+    layer = SparseGlobalAttention(B, H, N, device=dev)
+    layer.load_output_projection(wl.w_o)
+    layer.forward(*tail, wl.method, wl.budgets, wl.keep_k, wl.dense_q, wl.rounds, wl.rho,
+                  wl.eps, wl.select_seed)
+    out_view = torch.empty_like(layer.out)
+    R.ress_token_gather(shape, V, S, True, layer.out, out_view)
+    torch.cuda.synchronize()
+    assert torch.equal(tail[0], wl.q) and torch.equal(tail[2], wl.v)
+    assert torch.equal(out_view, ref.out[:, :, pos])
+
+
 def test_wide_logit_range_and_rescaling():
     """Logits spread over hundreds of units (Q scaled by 12): exp2 arguments reach the
     clamp at -126, the running max jumps between tiles and forces O rescales; a ragged
