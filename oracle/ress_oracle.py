@@ -391,14 +391,16 @@ def select_blocks(method: int, P, budgets: Sequence[int], keep_k=None, dense_q=N
 # attention").
 # ----------------------------------------------------------------------------------------
 def attention_qblock(q, k, v, b: int, h: int, i: int, kept: Sequence[int], scale: float,
-                     block: int = 128, dtype=np.float32):
-    """Output rows and natural-log LSE of query block i of head (b, h) attending to the
-    tokens of the kept key blocks (ascending blocks, tokens in order); tokens >= N do not
-    exist.  With no kept block the rows are zero and the LSE is -inf."""
+                     block: int = 128, dtype=np.float32, key_block: Optional[int] = None):
+    """Output rows and natural-log LSE of query block i (`block` tokens) of head (b, h)
+    attending to the tokens of the kept key blocks (`key_block` tokens each, default
+    `block`; ascending blocks, tokens in order); tokens >= N do not exist.  With no kept
+    block the rows are zero and the LSE is -inf."""
     N = q.shape[2]
+    kb = block if key_block is None else key_block
     r0, r1 = i * block, min(N, (i + 1) * block)
     rows = np.asarray(q[b, h, r0:r1], dtype=dtype)
-    idx = [t for j in kept for t in range(j * block, min(N, (j + 1) * block))]
+    idx = [t for j in kept for t in range(j * kb, min(N, (j + 1) * kb))]
     if not idx:
         return np.zeros((r1 - r0, q.shape[3]), dtype), np.full(r1 - r0, -np.inf, dtype)
     kk = np.asarray(k[b, h, idx], dtype=dtype)
@@ -413,11 +415,12 @@ def attention_qblock(q, k, v, b: int, h: int, i: int, kept: Sequence[int], scale
 
 
 def block_sparse_attn(q, k, v, kept: dict, scale: float, rows=None, block: int = 128,
-                      dtype=np.float32):
+                      dtype=np.float32, key_block: Optional[int] = None):
     """Attention for the query blocks in `rows` (default: every key of `kept`).
     Returns {(b,h,i): (out rows, lse)}."""
     rows = sorted(kept) if rows is None else rows
-    return {r: attention_qblock(q, k, v, *r, kept=kept[r], scale=scale, block=block, dtype=dtype)
+    return {r: attention_qblock(q, k, v, *r, kept=kept[r], scale=scale, block=block, dtype=dtype,
+                                key_block=key_block)
             for r in rows}
 
 
@@ -430,19 +433,22 @@ def to_numpy_f32(t) -> np.ndarray:
 
 def layer(q, k, v, w_o, method: int, budgets, keep_k=None, dense_q=None, rounds: int = 0,
           rho: float = 0.5, eps: float = 1e-4, seed: int = 0, rows=None,
-          attn_rows=None, block: int = 128, top_p: float = 1.0) -> dict:
+          attn_rows=None, block: int = 128, top_p: float = 1.0,
+          key_block: Optional[int] = None) -> dict:
     """The whole path for one layer: pool -> P, vbar -> drift -> select -> attention.
-    `rows` limits drift and selection to those (b,h,i); `attn_rows` limits the attention
-    (default: the selected rows)."""
+    Query blocks hold `block` tokens, key blocks `key_block` (default `block`; the pages'
+    grid is 128 x 64, [ReSS] Supp. F).  `rows` limits drift and selection to those
+    (b,h,i); `attn_rows` limits the attention (default: the selected rows)."""
     qf, kf, vf = to_numpy_f32(q), to_numpy_f32(k), to_numpy_f32(v)
     B, H, N, Dh = qf.shape
+    kb = block if key_block is None else key_block
     scale = 1.0 / math.sqrt(Dh)
-    qp, kp, vp = pool_blocks(qf, block), pool_blocks(kf, block), pool_blocks(vf, block)
+    qp, kp, vp = pool_blocks(qf, block), pool_blocks(kf, kb), pool_blocks(vf, kb)
     P, vbar = block_scores(qp, kp, vp, scale)
     gram = head_gram(to_numpy_f32(w_o), H, Dh)
-    nb = P.shape[-1]
+    nq = P.shape[-2]
     if rows is None:
-        rows = [(b, h, i) for b in range(B) for h in range(H) for i in range(nb)]
+        rows = [(b, h, i) for b in range(B) for h in range(H) for i in range(nq)]
     s = None
     if method == DRIFT:
         s = np.zeros_like(P)
@@ -452,6 +458,7 @@ def layer(q, k, v, w_o, method: int, budgets, keep_k=None, dense_q=None, rounds:
                         gram=gram, rounds=rounds, rho=rho, eps=eps, seed=seed, rows=rows,
                         top_p=top_p)
     attn = block_sparse_attn(qf, kf, vf, sel["kept"], scale,
-                             rows=rows if attn_rows is None else attn_rows, block=block)
+                             rows=rows if attn_rows is None else attn_rows, block=block,
+                             key_block=kb)
     return dict(q_pool=qp, k_pool=kp, v_pool=vp, P=P, vbar=vbar, gram=gram, s=s,
                 kept=sel["kept"], margin=sel["margin"], info=sel["info"], attn=attn)

@@ -77,3 +77,31 @@ def test_no_kept_block_gives_zero_rows():
     q, k, v = _qkv(4, N=256)
     o, l = O.attention_qblock(q.numpy(), k.numpy(), v.numpy(), 0, 0, 0, [], 0.125)
     assert np.all(o == 0) and np.all(np.isneginf(l))
+
+
+# ------------------------------------------- the pages' grid: key blocks of 64 tokens
+def test_key_blocks_of_64_pool_and_attend_like_their_pairs():
+    """[ReSS] Supp. F grid (query blocks of 128, key blocks of 64): two consecutive 64-token
+    pools average to the 128-token pool, and keeping both 64-blocks of a pair attends
+    exactly like keeping the 128-block that holds them."""
+    rng = np.random.default_rng(8)
+    N = 700                                        # 6 query blocks, 11 key blocks of 64
+    q, k, v = (rng.normal(size=(1, 2, N, 64)).astype(np.float32) for _ in range(3))
+    p128 = O.pool_blocks(k, 128, dtype=np.float64)
+    p64 = O.pool_blocks(k, 64, dtype=np.float64)
+    for j in range(5):                             # full 128-blocks
+        assert np.allclose(p128[:, :, j], 0.5 * (p64[:, :, 2 * j] + p64[:, :, 2 * j + 1]), atol=1e-12)
+    # last 128-block: 60 tokens = one partial 64-block
+    assert np.allclose(p128[:, :, 5], p64[:, :, 10], atol=1e-12)
+    for i in range(6):
+        kept128 = [0, 2, 5]
+        kept64 = [0, 1, 4, 5, 10]
+        o1, l1 = O.attention_qblock(q, k, v, 0, 1, i, kept128, 0.125, dtype=np.float64)
+        o2, l2 = O.attention_qblock(q, k, v, 0, 1, i, kept64, 0.125, dtype=np.float64,
+                                    key_block=64)
+        assert np.allclose(o1, o2, atol=1e-12) and np.allclose(l1, l2, atol=1e-12)
+    # a single 64-block is half of its 128-block: brute force against a direct softmax
+    o3, _ = O.attention_qblock(q, k, v, 0, 0, 2, [3], 0.125, dtype=np.float64, key_block=64)
+    lg = q[0, 0, 256:384].astype(np.float64) @ k[0, 0, 192:256].astype(np.float64).T * 0.125
+    pr = np.exp(lg - lg.max(1, keepdims=True))
+    assert np.allclose(o3, (pr / pr.sum(1, keepdims=True)) @ v[0, 0, 192:256], atol=1e-12)
