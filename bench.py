@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--top-p", type=float, default=0.9,
                     help="mass threshold of the cdf method (the budget from --sparsity caps it)")
     ap.add_argument("--sparsity", type=float, default=None)
+    ap.add_argument("--key-block", type=int, choices=[128, 64], default=128,
+                    help="tokens per key block (query blocks are 128); 64 = ReSS Supp. F grid")
     ap.add_argument("--objective", choices=["min", "max-swaps", "max-full"], default="min",
                     help="drift objective: the method, or a drift-maximising control (drift only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -139,21 +141,27 @@ class ClockSampler:
 def build_case(args, rank: int):
     from block_sparse_global_b200 import workload as W
     return W.make_workload(args.case, layer=rank, device="cuda", method=args.method,
-                           sparsity=args.sparsity)
+                           sparsity=args.sparsity, key_block=getattr(args, "key_block", 128))
 
 
-def kept_tile_flops(kv_idx, kv_cnt, N: int) -> float:
-    """Algorithmic FLOPs over kept tiles: sum of 4 * rows * cols * 64 (QK^T and PV), rows
-    and cols counting only tokens < N."""
+def workload_name(wl) -> str:
+    return wl.case.name + ("" if wl.key_block == 128 else f"-kb{wl.key_block}")
+
+
+def kept_tile_flops(kv_idx, kv_cnt, N: int, key_block: int = 128) -> float:
+    """Algorithmic FLOPs over the kept (query block, key block) pairs: sum of
+    4 * rows * cols * 64 (QK^T and PV), rows and cols counting only tokens < N (query
+    blocks of 128 tokens, key blocks of key_block)."""
     import torch
-    B, H, nb, _ = kv_idx.shape
-    ar = torch.arange(nb, device=kv_idx.device)
-    valid = torch.clamp(N - ar * 128, max=128).to(torch.float64)          # tokens per block
-    pos = torch.arange(nb, device=kv_idx.device).view(1, 1, 1, nb)
+    B, H, nq, nk = kv_idx.shape
+    dev = kv_idx.device
+    rows = torch.clamp(N - torch.arange(nq, device=dev) * 128, max=128).to(torch.float64)
+    valid = torch.clamp(N - torch.arange(nk, device=dev) * key_block, max=key_block).to(torch.float64)
+    pos = torch.arange(nk, device=dev).view(1, 1, 1, nk)
     live = pos < kv_cnt.unsqueeze(-1)
-    cols = torch.where(live, valid[kv_idx.clamp(0, nb - 1).long()], torch.zeros((), dtype=torch.float64,
-                                                                             device=kv_idx.device))
-    per_row = cols.sum(-1) * valid.view(1, 1, nb)
+    cols = torch.where(live, valid[kv_idx.clamp(0, nk - 1).long()],
+                       torch.zeros((), dtype=torch.float64, device=dev))
+    per_row = cols.sum(-1) * rows.view(1, 1, nq)
     return float(per_row.sum().item()) * 4.0 * 64.0
 
 
@@ -204,7 +212,7 @@ def run_ours(args):
     Bsz, H, N, _ = wl.q.shape
     q, k, v = wl.q, wl.k, wl.v
     keep_k, dense_q = wl.keep_k, wl.dense_q
-    layer = SparseGlobalAttention(Bsz, H, N, device=dev)
+    layer = SparseGlobalAttention(Bsz, H, N, device=dev, key_block=wl.key_block)
     layer.load_output_projection(wl.w_o)
     flush = torch.empty(L2_FLUSH_BYTES // 4, device=dev, dtype=torch.float32)
     stream = torch.cuda.current_stream()
@@ -234,11 +242,11 @@ def run_ours(args):
     torch.cuda.synchronize()
     if layer.device_error():
         raise SystemExit(f"device error {layer.device_error()} during warm-up")
-    flops = kept_tile_flops(layer.kv_idx, layer.kv_cnt, N)
-    kept_frac = float(layer.kv_cnt.sum().item()) / (Bsz * H * layer.nb * layer.nb)
+    flops = kept_tile_flops(layer.kv_idx, layer.kv_cnt, N, wl.key_block)
+    kept_frac = float(layer.kv_cnt.sum().item()) / (Bsz * H * layer.nq * layer.nk)
     # realized drift J of every row's selection (extra, untimed passes: the block map
     # written out, then the selection with its J output)
-    J = torch.zeros(Bsz, H, layer.nb, device=dev)
+    J = torch.zeros(Bsz, H, layer.nq, device=dev)
     layer.scores(q, k, v)
     layer.select(wl.method, wl.budgets, keep_k, dense_q, wl.rounds, wl.rho, wl.eps, wl.select_seed,
                  objective=objective, drift_out=J, top_p=args.top_p)
@@ -302,8 +310,9 @@ def run_ours(args):
             per[name] = round(statistics.median(times), 4)
         extra["kernels_ms"] = per
         # same-shape dense attention: every query block keeps every key block
-        dense_idx = torch.arange(layer.nb, device=dev, dtype=torch.int32).expand(Bsz, H, layer.nb, layer.nb).contiguous()
-        dense_cnt = torch.full((Bsz, H, layer.nb), layer.nb, device=dev, dtype=torch.int32)
+        nq, nk = layer.nq, layer.nk
+        dense_idx = torch.arange(nk, device=dev, dtype=torch.int32).expand(Bsz, H, nq, nk).contiguous()
+        dense_cnt = torch.full((Bsz, H, nq), nk, device=dev, dtype=torch.int32)
         dense_out = torch.empty_like(layer.out)
         dts = []
         for _ in range(5):
@@ -314,7 +323,7 @@ def run_ours(args):
             b.record(stream)
             torch.cuda.synchronize()
             dts.append(a.elapsed_time(b))
-        dense_flops = kept_tile_flops(dense_idx, dense_cnt, N)
+        dense_flops = kept_tile_flops(dense_idx, dense_cnt, N, wl.key_block)
         dms = statistics.median(dts)
         extra["dense_attention"] = {"ms": round(dms, 4), "tflops": round(dense_flops / dms / 1e9, 1)}
         del dense_idx, dense_cnt, dense_out
@@ -360,8 +369,8 @@ def run_ours(args):
         "dtype": "bf16",
         "data": "synthetic (seeded, VGGT-shaped)",
         "config": {
-            "workload": wl.case.name, "batch": Bsz, "heads": H, "seq_len": N, "head_dim": 64,
-            "block": 128, "method": ["mass", "drift", "random", "cdf"][wl.method], "sparsity": wl.sparsity,
+            "workload": workload_name(wl), "batch": Bsz, "heads": H, "seq_len": N, "head_dim": 64,
+            "block": 128, "key_block": wl.key_block, "method": ["mass", "drift", "random", "cdf"][wl.method], "sparsity": wl.sparsity,
             "rounds": wl.rounds, "budgets": sorted(set(wl.budgets)) if len(set(wl.budgets)) < 4 else "dirichlet",
             "drift_objective": args.objective, "realized_drift_J_mean": float(f"{drift_mean:.6g}"),
             **({"top_p": args.top_p} if wl.method == R.SELECT_CDF else {}),
@@ -372,7 +381,7 @@ def run_ours(args):
         "roofline": {"kernel": "block_sparse_attn", "bound": "tensor", "achieved": round(achieved, 2),
                      "peak": bf16_peak, "unit": "TFLOP/s", "frac": round(achieved / bf16_peak, 4),
                      "peak_source": f"{peak_kind} dense bf16 (burst)",
-                     "traffic": measured_traffic(wl.case.name), "traffic_unit": "bytes per launch (ncu)",
+                     "traffic": measured_traffic(workload_name(wl)), "traffic_unit": "bytes per launch (ncu)",
                      "mean_launch_ms": round(attn_mean, 4)},
         "gpu_launches": args.steps * layer.kernel_launches(wl.method),
     }
@@ -405,11 +414,13 @@ def _oracle_sample(wl, heads, top_p: float = 1.0):
     budgets = [wl.budgets[h] for h in heads]
     t0 = time.perf_counter()
     res = O.layer(q, k, v, w_o, wl.method, budgets, wl.keep_k.cpu().numpy(), wl.dense_q.cpu().numpy(),
-                  rounds=wl.rounds, rho=wl.rho, eps=wl.eps, seed=wl.select_seed, top_p=top_p)
+                  rounds=wl.rounds, rho=wl.rho, eps=wl.eps, seed=wl.select_seed, top_p=top_p,
+                  key_block=wl.key_block)
     dt = time.perf_counter() - t0
-    N = q.shape[2]
-    valid = [min(128, N - 128 * j) for j in range((N + 127) // 128)]
-    fl = sum(4.0 * 64 * valid[i] * sum(valid[j] for j in kept) for (b, h, i), kept in res["kept"].items())
+    N, kb = q.shape[2], wl.key_block
+    rows = [min(128, N - 128 * i) for i in range((N + 127) // 128)]
+    valid = [min(kb, N - kb * j) for j in range((N + kb - 1) // kb)]
+    fl = sum(4.0 * 64 * rows[i] * sum(valid[j] for j in kept) for (b, h, i), kept in res["kept"].items())
     return dt, fl
 
 
@@ -445,7 +456,8 @@ def run_reference(args):
         return
     import torch
     from block_sparse_global_b200 import workload as W
-    wl = W.make_workload(args.case, layer=0, device="cpu", method=args.method, sparsity=args.sparsity)
+    wl = W.make_workload(args.case, layer=0, device="cpu", method=args.method, sparsity=args.sparsity,
+                         key_block=getattr(args, "key_block", 128))
     H = wl.q.shape[1]
     times, flops = [], []
     for s in range(args.warmup + args.steps):
@@ -459,8 +471,8 @@ def run_reference(args):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1e3 * statistics.mean(times), 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded, VGGT-shaped)",
-        "config": {"workload": wl.case.name, "batch": 1, "heads": H, "seq_len": wl.q.shape[2],
-                   "head_dim": 64, "block": 128, "method": ["mass", "drift", "random", "cdf"][wl.method],
+        "config": {"workload": workload_name(wl), "batch": 1, "heads": H, "seq_len": wl.q.shape[2],
+                   "head_dim": 64, "block": 128, "key_block": wl.key_block, "method": ["mass", "drift", "random", "cdf"][wl.method],
                    "sparsity": wl.sparsity, "rounds": wl.rounds,
                    "step": "oracle whole path for one head of the layer (heads rotate)"},
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",

@@ -3,7 +3,11 @@
 // [ReSS] = "ReSS: Residual-Restoring Sparse Attention for 3D Vision Transformers",
 // §3 step (3): exact attention over the kept key blocks, softmax renormalised among
 // them.  One CTA computes one (batch, head, query block) row of 128 queries against the
-// key blocks listed in kv_idx; two CTAs share an SM.
+// key blocks listed in kv_idx; two CTAs share an SM.  Key blocks are 128 tokens (one
+// block per 128 x 128 score tile) or 64 tokens, the grid of ReSS Supp. F: then kept
+// blocks 2j and 2j+1 of a row fill the two 64-row halves of tile j, each through its own
+// 64-row TMA box, and an odd count leaves the second half of the last tile zero (a box
+// that starts past the last token) and masked.
 //
 // Warp roles (192 threads):
 //   warps 0-3  softmax: thread t owns query row t (tensor-memory lane t).  Reads the
@@ -138,11 +142,13 @@ struct AttnParams {
   __nv_bfloat16 *out;
   float *lse;
   int32_t *dev_err;
-  int N, nb;
+  int N, nq, nk;  // tokens; query and key blocks per (batch, head)
   long long items;
   float scale_log2;
 };
 
+// KB = tokens per key block (128 or 64); a score tile always spans 128 keys.
+template <int KB>
 __global__ void __launch_bounds__(kThreads, 2)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ AttnParams p) {
@@ -153,10 +159,12 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   const long long item = p.order ? (long long)p.order[blockIdx.x] : (long long)blockIdx.x;
-  const long long bh = item / p.nb;
-  const int qi = (int)(item - bh * p.nb);
+  const long long bh = item / p.nq;
+  const int qi = (int)(item - bh * p.nq);
   const int cnt = p.kv_cnt[item];
-  const int32_t *kvrow = p.kv_idx + item * p.nb;
+  const int32_t *kvrow = p.kv_idx + item * p.nk;
+  // score tiles of the row: one per kept block, or one per pair of 64-token blocks
+  const int tiles = KB == 128 ? cnt : (cnt + 1) >> 1;
 
   if (tid == 0) {
     mbar_init(&bar->q_full, 1);
@@ -177,12 +185,12 @@ __global__ void __launch_bounds__(kThreads, 2)
     fence_mbar_init();
   }
   if (warp == kProducerWarp) {
-    // validate the row before any work: count in range, every entry in [0, nb)
-    bool bad = cnt < 0 || cnt > p.nb;
+    // validate the row before any work: count in range, every entry in [0, nk)
+    bool bad = cnt < 0 || cnt > p.nk;
     if (!bad)
       for (int j = lane; j < cnt; j += 32) {
         const int kb = kvrow[j];
-        bad |= kb < 0 || kb >= p.nb;
+        bad |= kb < 0 || kb >= p.nk;
       }
     bad = __any_sync(0xffffffffu, bad);
     if (lane == 0) bar->row_state = bad ? 2 : (cnt == 0 ? 1 : 0);
@@ -211,32 +219,42 @@ __global__ void __launch_bounds__(kThreads, 2)
         tma_prefetch_desc(&tmV);
         mbar_arrive_expect_tx(&bar->q_full, kTile);
         tma_load_3d(smem + kOffQ, &tmQ, &bar->q_full, 0, qi * 128, (int)bh);
+        // tile j into one ring slot: one 128-row box, or two 64-row boxes (kept blocks
+        // 2j and 2j+1; row N, past the last token, reads as zero when 2j+1 == cnt)
+        auto load_tile = [&](const CUtensorMap *tm, unsigned char *dst, uint64_t *full, int j) {
+          mbar_arrive_expect_tx(full, kTile);
+          if constexpr (KB == 128) {
+            tma_load_3d(dst, tm, full, 0, kvrow[j] * 128, (int)bh);
+          } else {
+            const int r1 = 2 * j + 1 < cnt ? kvrow[2 * j + 1] * 64 : p.N;
+            tma_load_3d(dst, tm, full, 0, kvrow[2 * j] * 64, (int)bh);
+            tma_load_3d(dst + kTile / 2, tm, full, 0, r1, (int)bh);
+          }
+        };
         auto load_k = [&](int j) {
           const int s = j % kKStages;
-          mbar_arrive_expect_tx(&bar->k_full[s], kTile);
-          tma_load_3d(smem + kOffK + s * kTile, &tmK, &bar->k_full[s], 0, kvrow[j] * 128, (int)bh);
+          load_tile(&tmK, smem + kOffK + s * kTile, &bar->k_full[s], j);
         };
         auto load_v = [&](int j) {
           const int s = j % kVStages;
-          mbar_arrive_expect_tx(&bar->v_full[s], kTile);
-          tma_load_3d(smem + kOffV + s * kTile, &tmV, &bar->v_full[s], 0, kvrow[j] * 128, (int)bh);
+          load_tile(&tmV, smem + kOffV + s * kTile, &bar->v_full[s], j);
         };
-        int nk = min(cnt, kKStages), nv = min(cnt, kVStages);
+        int nk = min(tiles, kKStages), nv = min(tiles, kVStages);
         for (int j = 0; j < nk; ++j) load_k(j);
         for (int j = 0; j < nv; ++j) load_v(j);
-        for (int j = 0; j < cnt; ++j) {
-          if (j + kKStages < cnt) {
+        for (int j = 0; j < tiles; ++j) {
+          if (j + kKStages < tiles) {
             if (!mbar_wait(&bar->k_empty[j % kKStages], (j / kKStages) & 1, abort)) break;
             load_k(j + kKStages);
             nk = j + kKStages + 1;
           }
-          if (j + kVStages < cnt) {
+          if (j + kVStages < tiles) {
             if (!mbar_wait(&bar->v_empty[j % kVStages], (j / kVStages) & 1, abort)) break;
             load_v(j + kVStages);
             nv = j + kVStages + 1;
           }
         }
-        if (*abort == 0 && (nk < cnt || nv < cnt)) {
+        if (*abort == 0 && (nk < tiles || nv < tiles)) {
           report_error(p.dev_err, RESS_ERR_DEVICE_TIMEOUT);
           *abort = 1;
         }
@@ -256,8 +274,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         bool ok = mbar_wait(&bar->q_full, 0, abort);
         tc_fence_after();
         const uint64_t dq = smem_desc(sQ);
-        for (int j = 0; ok && j <= cnt; ++j) {
-          if (j < cnt) {
+        for (int j = 0; ok && j <= tiles; ++j) {
+          if (j < tiles) {
             const int s = j % kKStages;
             ok = mbar_wait(&bar->k_full[s], (j / kKStages) & 1, abort);
             if (ok && j > 0) ok = mbar_wait(&bar->s_free, (j - 1) & 1, abort);
@@ -295,13 +313,20 @@ __global__ void __launch_bounds__(kThreads, 2)
       // ------------------------------------------------------------- softmax
       const int row = tid;  // 0..127, tensor-memory lane
       const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
-      const int last_valid = p.N - (p.nb - 1) * 128;  // tokens in the last block
+      const int last_valid = p.N - (p.nk - 1) * KB;  // tokens in the last key block
       float m_run = -INFINITY, l_run = 0.f;
       bool ok = true;
+      // kept block(s) of the next tile, read ahead of the barrier wait
       int kb_next = kvrow[0];
-      for (int j = 0; j < cnt && ok; ++j) {
-        const int kb = kb_next;
-        if (j + 1 < cnt) kb_next = kvrow[j + 1];
+      int kb2_next = KB == 64 ? (cnt > 1 ? kvrow[1] : -1) : -1;
+      for (int j = 0; j < tiles && ok; ++j) {
+        const int kb = kb_next, kb2 = kb2_next;
+        if constexpr (KB == 128) {
+          if (j + 1 < tiles) kb_next = kvrow[j + 1];
+        } else {
+          if (2 * j + 2 < cnt) kb_next = kvrow[2 * j + 2];
+          kb2_next = 2 * j + 3 < cnt ? kvrow[2 * j + 3] : -1;
+        }
         ok = mbar_wait(&bar->s_full, j & 1, abort);
         if (!ok) break;
         tc_fence_after();
@@ -313,10 +338,24 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar->s_free);
-        if (kb == p.nb - 1 && last_valid < 128) {
+        if constexpr (KB == 128) {
+          if (kb == p.nk - 1 && last_valid < 128) {
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (c >= last_valid) sv[c] = __float_as_uint(-INFINITY);
+            for (int c = 0; c < 128; ++c)
+              if (c >= last_valid) sv[c] = __float_as_uint(-INFINITY);
+          }
+        } else {
+          // valid keys in each 64-column half: the last block is ragged, an absent
+          // second block has none
+          const int lim0 = kb == p.nk - 1 ? last_valid : 64;
+          const int lim1 = kb2 < 0 ? 0 : (kb2 == p.nk - 1 ? last_valid : 64);
+          if (lim0 < 64 || lim1 < 64) {
+#pragma unroll
+            for (int c = 0; c < 64; ++c) {
+              if (c >= lim0) sv[c] = __float_as_uint(-INFINITY);
+              if (c >= lim1) sv[64 + c] = __float_as_uint(-INFINITY);
+            }
+          }
         }
         // row max: four chains of 3-input max
         float mc[4];
@@ -378,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (lane == 0) mbar_arrive(&bar->p_full);
         m_run = m_use;
       }
-      if (ok) ok = mbar_wait(&bar->o_done, (cnt - 1) & 1, abort);
+      if (ok) ok = mbar_wait(&bar->o_done, (tiles - 1) & 1, abort);
       if (!ok) {
         report_error(p.dev_err, RESS_ERR_DEVICE_TIMEOUT);
         *abort = 1;
@@ -435,14 +474,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [B*H, N, 64] bf16 viewed as a 3-D tensor (64, N, B*H); box (64, 128, 1); rows past N
+// [B*H, N, 64] bf16 viewed as a 3-D tensor (64, N, B*H); box (64, rows, 1); rows past N
 // read as zero.
-bool make_map(CUtensorMap *m, const void *base, int N, long long BH) {
+bool make_map(CUtensorMap *m, const void *base, int N, long long BH, int rows) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {64, (cuuint64_t)N, (cuuint64_t)BH};
   cuuint64_t strides[2] = {128, (cuuint64_t)N * 128};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -454,8 +493,8 @@ bool make_map(CUtensorMap *m, const void *base, int N, long long BH) {
 
 cudaError_t launch_attn(const Dims &d, const AttnLaunch &a, cudaStream_t st) {
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, a.q, d.N, d.BH()) || !make_map(&mk, a.k, d.N, d.BH()) ||
-      !make_map(&mv, a.v, d.N, d.BH()))
+  if (!make_map(&mq, a.q, d.N, d.BH(), 128) || !make_map(&mk, a.k, d.N, d.BH(), d.kb) ||
+      !make_map(&mv, a.v, d.N, d.BH(), d.kb))
     return cudaErrorNotSupported;
   AttnParams p;
   p.kv_idx = a.kv_idx;
@@ -465,13 +504,15 @@ cudaError_t launch_attn(const Dims &d, const AttnLaunch &a, cudaStream_t st) {
   p.lse = a.lse;
   p.dev_err = a.dev_err;
   p.N = d.N;
-  p.nb = d.nb;
-  p.items = d.BH() * d.nb;
+  p.nq = d.nq;
+  p.nk = d.nk;
+  p.items = d.BH() * d.nq;
   p.scale_log2 = a.scale * 1.4426950408889634f;
+  auto kern = d.kb == 64 ? attn_kernel<64> : attn_kernel<128>;
   cudaError_t e =
-      cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  attn_kernel<<<(unsigned)p.items, kThreads, kSmemBytes, st>>>(mq, mk, mv, p);
+  kern<<<(unsigned)p.items, kThreads, kSmemBytes, st>>>(mq, mk, mv, p);
   return cudaGetLastError();
 }
 

@@ -72,20 +72,28 @@ __global__ void __launch_bounds__(kPoolWarps * 32) pool_kernel(const uint4 *__re
                                                                float *__restrict__ qp,
                                                                float *__restrict__ kp,
                                                                float *__restrict__ vp, long long BH,
-                                                               int N, int nb) {
+                                                               int N, int nq, int nk, int kb) {
   const int lane = threadIdx.x & 31;
   const int cg = lane & 7, ts = lane >> 3;
-  const long long per_tensor = BH * nb;
-  const long long units = 3 * per_tensor;
+  // queries are pooled over nq blocks of 128 tokens, keys and values over nk blocks of kb
+  const long long q_units = BH * nq, k_units = BH * nk;
+  const long long units = q_units + 2 * k_units;
   for (long long u = (long long)blockIdx.x * kPoolWarps + (threadIdx.x >> 5); u < units;
        u += (long long)gridDim.x * kPoolWarps) {
-    const int which = (int)(u / per_tensor);
-    const long long rem = u - which * per_tensor;
-    const long long bh = rem / nb;
-    const int j = (int)(rem - bh * nb);
+    int which, nbw, bw;
+    long long rem;
+    if (u < q_units) {
+      which = 0, rem = u, nbw = nq, bw = kBlock;
+    } else {
+      const long long r2 = u - q_units;
+      which = 1 + (int)(r2 / k_units);
+      rem = r2 - (which - 1) * k_units, nbw = nk, bw = kb;
+    }
+    const long long bh = rem / nbw;
+    const int j = (int)(rem - bh * nbw);
     const uint4 *src = (which == 0 ? q : which == 1 ? k : v) + (size_t)bh * N * 8;
-    float *dst = (which == 0 ? qp : which == 1 ? kp : vp) + ((size_t)bh * nb + j) * kHeadDim;
-    const int t0 = j * kBlock, t1 = min(N, t0 + kBlock);
+    float *dst = (which == 0 ? qp : which == 1 ? kp : vp) + ((size_t)bh * nbw + j) * kHeadDim;
+    const int t0 = j * bw, t1 = min(N, t0 + bw);
     float acc[8];
 #pragma unroll
     for (int c = 0; c < 8; ++c) acc[c] = 0.f;
@@ -178,7 +186,7 @@ __host__ __device__ __forceinline__ size_t fused_warp_bytes(int nb, bool cdf) {
 template <int TQ, bool SEL>
 __global__ void __launch_bounds__(kThreads) block_scores_kernel(
     const float *__restrict__ qp, const float *__restrict__ kp, const float *__restrict__ vp,
-    float scale, float *__restrict__ P, float *__restrict__ vbar, int nb,
+    float scale, float *__restrict__ P, float *__restrict__ vbar, int nq, int nk,
     const __grid_constant__ FusedSelect fs) {
   constexpr int R = TQ / kWarps;
   extern __shared__ __align__(16) float sm[];
@@ -188,13 +196,13 @@ __global__ void __launch_bounds__(kThreads) block_scores_kernel(
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const long long bh = blockIdx.y;
   const int i0 = blockIdx.x * TQ;
-  const float *qh = qp + (size_t)bh * nb * kHeadDim;
+  const float *qh = qp + (size_t)bh * nq * kHeadDim;
   for (int idx = t; idx < TQ * kHeadDim; idx += kThreads) {
     const int r = idx / kHeadDim;
-    sq[idx] = (i0 + r < nb) ? qh[(size_t)(i0 + r) * kHeadDim + idx % kHeadDim] : 0.f;
+    sq[idx] = (i0 + r < nq) ? qh[(size_t)(i0 + r) * kHeadDim + idx % kHeadDim] : 0.f;
   }
   // logits: lane takes key blocks lane and lane + 32 of each tile
-  tile_stream(tiles, kp + (size_t)bh * nb * kHeadDim, nb, [&](int tt, const float *tile) {
+  tile_stream(tiles, kp + (size_t)bh * nk * kHeadDim, nk, [&](int tt, const float *tile) {
     const float4 *k0 = reinterpret_cast<const float4 *>(tile + lane * kTilePad);
     const float4 *k1 = reinterpret_cast<const float4 *>(tile + (lane + 32) * kTilePad);
 #pragma unroll
@@ -209,28 +217,28 @@ __global__ void __launch_bounds__(kThreads) block_scores_kernel(
         a1 = fmaf(x.x, y1.x, a1); a1 = fmaf(x.y, y1.y, a1); a1 = fmaf(x.z, y1.z, a1); a1 = fmaf(x.w, y1.w, a1);
       }
       const int j = tt * kTileKeys + lane;
-      if (j < nb) sl[r * nb + j] = a0 * scale;
-      if (j + 32 < nb) sl[r * nb + j + 32] = a1 * scale;
+      if (j < nk) sl[r * nk + j] = a0 * scale;
+      if (j + 32 < nk) sl[r * nk + j + 32] = a1 * scale;
     }
   });
   // softmax over every key block, per row
 #pragma unroll
   for (int q = 0; q < R; ++q) {
     const int r = warp * R + q, i = i0 + r;
-    if (i >= nb) continue;
-    float *row = sl + r * nb;
+    if (i >= nq) continue;
+    float *row = sl + r * nk;
     float m = -INFINITY;
-    for (int j = lane; j < nb; j += 32) m = fmaxf(m, row[j]);
+    for (int j = lane; j < nk; j += 32) m = fmaxf(m, row[j]);
     m = warp_max(m);
     float sum = 0.f;
-    for (int j = lane; j < nb; j += 32) {
+    for (int j = lane; j < nk; j += 32) {
       const float e = expf(row[j] - m);
       row[j] = e;
       sum += e;
     }
     sum = warp_sum(sum);
-    float *prow = P ? P + ((size_t)bh * nb + i) * nb : nullptr;
-    for (int j = lane; j < nb; j += 32) {
+    float *prow = P ? P + ((size_t)bh * nq + i) * nk : nullptr;
+    for (int j = lane; j < nk; j += 32) {
       const float pj = __fdiv_rn(row[j], sum);
       row[j] = pj;
       if (prow) prow[j] = pj;
@@ -241,21 +249,21 @@ __global__ void __launch_bounds__(kThreads) block_scores_kernel(
     // the same decisions as the selection kernel: top-c of the candidates by P (or by
     // the SplitMix64 key), ties to the lower block index; dense rows keep every block
     const bool cdf = fs.method == RESS_SELECT_CDF;
-    unsigned char *wb = reinterpret_cast<unsigned char *>(sl + (size_t)TQ * nb) +
-                        fused_warp_bytes(nb, cdf) * warp;
+    unsigned char *wb = reinterpret_cast<unsigned char *>(sl + (size_t)TQ * nk) +
+                        fused_warp_bytes(nk, cdf) * warp;
     uint32_t *hist = reinterpret_cast<uint32_t *>(wb);
     int *slot = reinterpret_cast<int *>(wb + 1024);
     uint8_t *st = wb + 1152;
-    float *sorted = reinterpret_cast<float *>(st + ((nb + 15) & ~15));
+    float *sorted = reinterpret_cast<float *>(st + ((nk + 15) & ~15));
     const int h = (int)(bh % fs.H);
 #pragma unroll 1
     for (int q = 0; q < R; ++q) {
       const int r = warp * R + q, i = i0 + r;
-      if (i >= nb) continue;
-      const float *row = sl + r * nb;
+      if (i >= nq) continue;
+      const float *row = sl + r * nk;
       const bool dense = fs.dense_q != nullptr && fs.dense_q[i] != 0;
       int n_cand = 0;
-      for (int j = lane; j < nb; j += 32) {
+      for (int j = lane; j < nk; j += 32) {
         const bool fixed = fs.keep_k != nullptr && fs.keep_k[j] != 0;
         st[j] = fixed ? kFixed : kCand;
         n_cand += fixed ? 0 : 1;
@@ -267,34 +275,34 @@ __global__ void __launch_bounds__(kThreads) block_scores_kernel(
         auto is_cand = [&](int j) { return st[j] == kCand; };
         auto keep = [&](int j) { st[j] = kKept; };
         if (fs.method == RESS_SELECT_MASS || cdf) {
-          warp_select<uint32_t>(nb, c, [&](int j) { return float_key(row[j]); }, is_cand, keep, hist, slot);
+          warp_select<uint32_t>(nk, c, [&](int j) { return float_key(row[j]); }, is_cand, keep, hist, slot);
           if (cdf) {
             double fixed = 0.0;  // mass of the always-kept blocks
-            for (int j = lane; j < nb; j += 32)
+            for (int j = lane; j < nk; j += 32)
               if (st[j] == kFixed) fixed += (double)row[j];
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) fixed += __shfl_xor_sync(0xffffffffu, fixed, o);
-            warp_cdf_cut(nb, row, [&](int j) { return st[j] == kKept; }, [&](int j) { st[j] = kCand; },
+            warp_cdf_cut(nk, row, [&](int j) { return st[j] == kKept; }, [&](int j) { st[j] = kCand; },
                          fixed, fs.top_p, sorted);
           }
         } else {
-          const uint64_t base = ((uint64_t)bh * nb + (uint64_t)i) * (uint64_t)nb;
-          warp_select<uint64_t>(nb, c, [&](int j) { return splitmix64_key(fs.seed, base + (uint64_t)j + 1); },
+          const uint64_t base = ((uint64_t)bh * nq + (uint64_t)i) * (uint64_t)nk;
+          warp_select<uint64_t>(nk, c, [&](int j) { return splitmix64_key(fs.seed, base + (uint64_t)j + 1); },
                                is_cand, keep, hist, slot);
         }
       }
-      int32_t *out = fs.kv_idx + ((size_t)bh * nb + i) * nb;
-      uint8_t *mrow = fs.mask ? fs.mask + ((size_t)bh * nb + i) * nb : nullptr;
+      int32_t *out = fs.kv_idx + ((size_t)bh * nq + i) * nk;
+      uint8_t *mrow = fs.mask ? fs.mask + ((size_t)bh * nq + i) * nk : nullptr;
       int total = 0;
-      for (int base = 0; base < nb; base += 32) {
+      for (int base = 0; base < nk; base += 32) {
         const int j = base + lane;
-        const bool k = j < nb && (dense || st[j] != kCand);
+        const bool k = j < nk && (dense || st[j] != kCand);
         const unsigned bal = __ballot_sync(0xffffffffu, k);
         if (k) out[total + __popc(bal & lanemask_lt())] = j;
-        if (mrow && j < nb) mrow[j] = k ? 1 : 0;
+        if (mrow && j < nk) mrow[j] = k ? 1 : 0;
         total += __popc(bal);
       }
-      if (lane == 0) fs.kv_cnt[(size_t)bh * nb + i] = total;
+      if (lane == 0) fs.kv_cnt[(size_t)bh * nq + i] = total;
       __syncwarp();
     }
     if (vbar == nullptr) return;
@@ -303,11 +311,11 @@ __global__ void __launch_bounds__(kThreads) block_scores_kernel(
   float a0[R], a1[R];
 #pragma unroll
   for (int q = 0; q < R; ++q) a0[q] = a1[q] = 0.f;
-  tile_stream(tiles, vp + (size_t)bh * nb * kHeadDim, nb, [&](int tt, const float *tile) {
-    const int jn = min(kTileKeys, nb - tt * kTileKeys);
+  tile_stream(tiles, vp + (size_t)bh * nk * kHeadDim, nk, [&](int tt, const float *tile) {
+    const int jn = min(kTileKeys, nk - tt * kTileKeys);
 #pragma unroll
     for (int q = 0; q < R; ++q) {
-      const float *row = sl + (warp * R + q) * nb + tt * kTileKeys;
+      const float *row = sl + (warp * R + q) * nk + tt * kTileKeys;
       for (int kk = 0; kk < jn; ++kk) {
         const float pj = row[kk];
         a0[q] = fmaf(pj, tile[kk * kTilePad + lane], a0[q]);
@@ -318,8 +326,8 @@ __global__ void __launch_bounds__(kThreads) block_scores_kernel(
 #pragma unroll
   for (int q = 0; q < R; ++q) {
     const int i = i0 + warp * R + q;
-    if (i < nb) {
-      float *o = vbar + ((size_t)bh * nb + i) * kHeadDim;
+    if (i < nq) {
+      float *o = vbar + ((size_t)bh * nq + i) * kHeadDim;
       o[lane] = a0[q];
       o[lane + 32] = a1[q];
     }
@@ -332,7 +340,7 @@ __global__ void __launch_bounds__(kThreads) block_scores_kernel(
 // c_j = V_j^T M V_j in the workspace.
 __global__ void __launch_bounds__(kThreads) drift_prep_kernel(
     const float *__restrict__ vp, const float *__restrict__ vbar, const float *__restrict__ gram,
-    float *__restrict__ w, float *__restrict__ a, float *__restrict__ c, int H, int nb) {
+    float *__restrict__ w, float *__restrict__ a, float *__restrict__ c, int H, int nq, int nk) {
   __shared__ float sM[kHeadDim][kPad];
   __shared__ float sx[kWarps][kHeadDim];
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
@@ -342,8 +350,9 @@ __global__ void __launch_bounds__(kThreads) drift_prep_kernel(
   for (int idx = t; idx < kHeadDim * kHeadDim; idx += kThreads)
     sM[idx / kHeadDim][idx % kHeadDim] = gram[(size_t)h * kHeadDim * kHeadDim + idx];
   __syncthreads();
-  const float *src = (rows ? vbar : vp) + (size_t)bh * nb * kHeadDim;
-  for (int n = blockIdx.x * 32 + warp; n < min(nb, (int)blockIdx.x * 32 + 32); n += kWarps) {
+  const int cnt = rows ? nq : nk;  // vbar has nq rows, the pooled values nk
+  const float *src = (rows ? vbar : vp) + (size_t)bh * cnt * kHeadDim;
+  for (int n = blockIdx.x * 32 + warp; n < min(cnt, (int)blockIdx.x * 32 + 32); n += kWarps) {
     sx[warp][lane] = src[(size_t)n * kHeadDim + lane];
     sx[warp][lane + 32] = src[(size_t)n * kHeadDim + lane + 32];
     __syncwarp();
@@ -356,11 +365,11 @@ __global__ void __launch_bounds__(kThreads) drift_prep_kernel(
     }
     const float dot = warp_sum(sx[warp][lane] * y0 + sx[warp][lane + 32] * y1);
     if (rows) {
-      w[((size_t)bh * nb + n) * kHeadDim + lane] = y0;
-      w[((size_t)bh * nb + n) * kHeadDim + lane + 32] = y1;
-      if (lane == 0) a[(size_t)bh * nb + n] = dot;
+      w[((size_t)bh * nq + n) * kHeadDim + lane] = y0;
+      w[((size_t)bh * nq + n) * kHeadDim + lane + 32] = y1;
+      if (lane == 0) a[(size_t)bh * nq + n] = dot;
     } else if (lane == 0) {
-      c[(size_t)bh * nb + n] = dot;
+      c[(size_t)bh * nk + n] = dot;
     }
     __syncwarp();
   }
@@ -372,7 +381,7 @@ __global__ void __launch_bounds__(kThreads) drift_prep_kernel(
 constexpr int kDriftRows = 16;
 __global__ void __launch_bounds__(kThreads) drift_kernel(
     const float *__restrict__ P, const float *__restrict__ vp, const float *__restrict__ w,
-    const float *__restrict__ a, const float *__restrict__ c, float *__restrict__ s, int nb) {
+    const float *__restrict__ a, const float *__restrict__ c, float *__restrict__ s, int nq, int nk) {
   constexpr int R = kDriftRows / kWarps;
   __shared__ __align__(16) float tiles[2 * kTileFloats];
   __shared__ __align__(16) float sw[kDriftRows][kHeadDim];
@@ -381,20 +390,20 @@ __global__ void __launch_bounds__(kThreads) drift_kernel(
   const int i0 = blockIdx.x * kDriftRows;
   for (int idx = t; idx < kDriftRows * kHeadDim; idx += kThreads) {
     const int r = idx / kHeadDim;
-    sw[r][idx % kHeadDim] = (i0 + r < nb) ? w[((size_t)bh * nb + i0 + r) * kHeadDim + idx % kHeadDim] : 0.f;
+    sw[r][idx % kHeadDim] = (i0 + r < nq) ? w[((size_t)bh * nq + i0 + r) * kHeadDim + idx % kHeadDim] : 0.f;
   }
   float ai[R];
 #pragma unroll
   for (int q = 0; q < R; ++q) {
     const int i = i0 + warp * R + q;
-    ai[q] = i < nb ? a[(size_t)bh * nb + i] : 0.f;
+    ai[q] = i < nq ? a[(size_t)bh * nq + i] : 0.f;
   }
-  const float *ch = c + (size_t)bh * nb;
-  tile_stream(tiles, vp + (size_t)bh * nb * kHeadDim, nb, [&](int tt, const float *tile) {
+  const float *ch = c + (size_t)bh * nk;
+  tile_stream(tiles, vp + (size_t)bh * nk * kHeadDim, nk, [&](int tt, const float *tile) {
     const float4 *v0 = reinterpret_cast<const float4 *>(tile + lane * kTilePad);
     const float4 *v1 = reinterpret_cast<const float4 *>(tile + (lane + 32) * kTilePad);
     const int j0 = tt * kTileKeys + lane, j1 = j0 + 32;
-    const float c0 = j0 < nb ? ch[j0] : 0.f, c1 = j1 < nb ? ch[j1] : 0.f;
+    const float c0 = j0 < nk ? ch[j0] : 0.f, c1 = j1 < nk ? ch[j1] : 0.f;
 #pragma unroll
     for (int q = 0; q < R; ++q) {
       const int r = warp * R + q, i = i0 + r;
@@ -406,10 +415,10 @@ __global__ void __launch_bounds__(kThreads) drift_kernel(
         d0 = fmaf(x.x, y0.x, d0); d0 = fmaf(x.y, y0.y, d0); d0 = fmaf(x.z, y0.z, d0); d0 = fmaf(x.w, y0.w, d0);
         d1 = fmaf(x.x, y1.x, d1); d1 = fmaf(x.y, y1.y, d1); d1 = fmaf(x.z, y1.z, d1); d1 = fmaf(x.w, y1.w, d1);
       }
-      if (i < nb) {
-        const size_t o = ((size_t)bh * nb + i) * nb;
-        if (j0 < nb) s[o + j0] = P[o + j0] * sqrtf(fmaxf((ai[q] - 2.f * d0) + c0, 0.f));
-        if (j1 < nb) s[o + j1] = P[o + j1] * sqrtf(fmaxf((ai[q] - 2.f * d1) + c1, 0.f));
+      if (i < nq) {
+        const size_t o = ((size_t)bh * nq + i) * nk;
+        if (j0 < nk) s[o + j0] = P[o + j0] * sqrtf(fmaxf((ai[q] - 2.f * d0) + c0, 0.f));
+        if (j1 < nk) s[o + j1] = P[o + j1] * sqrtf(fmaxf((ai[q] - 2.f * d1) + c1, 0.f));
       }
     }
   });
@@ -435,12 +444,12 @@ cudaError_t launch_token_gather(const Dims &d, int views, int specials, bool inv
 
 cudaError_t launch_pool(const Dims &d, const void *q, const void *k, const void *v, float *qp,
                         float *kp, float *vp, cudaStream_t st) {
-  const long long units = 3 * d.BH() * d.nb;
+  const long long units = d.BH() * d.nq + 2 * d.BH() * d.nk;
   long long blocks = (units + kPoolWarps - 1) / kPoolWarps;
   if (blocks > 148 * 256) blocks = 148 * 256;
   pool_kernel<<<(unsigned)blocks, kPoolWarps * 32, 0, st>>>(
       static_cast<const uint4 *>(q), static_cast<const uint4 *>(k), static_cast<const uint4 *>(v),
-      qp, kp, vp, d.BH(), d.N, d.nb);
+      qp, kp, vp, d.BH(), d.N, d.nq, d.nk, d.kb);
   return cudaGetLastError();
 }
 
@@ -448,13 +457,13 @@ template <int TQ, bool SEL>
 static cudaError_t scores_tq(const Dims &d, const float *qp, const float *kp, const float *vp,
                              float scale, float *P, float *vbar, const FusedSelect &fs,
                              cudaStream_t st) {
-  const size_t smem = sizeof(float) * (2 * kTileFloats + TQ * kHeadDim + (size_t)TQ * d.nb) +
-                      (SEL ? fused_warp_bytes(d.nb, fs.method == RESS_SELECT_CDF) * kWarps : 0);
+  const size_t smem = sizeof(float) * (2 * kTileFloats + TQ * kHeadDim + (size_t)TQ * d.nk) +
+                      (SEL ? fused_warp_bytes(d.nk, fs.method == RESS_SELECT_CDF) * kWarps : 0);
   cudaError_t e = cudaFuncSetAttribute(block_scores_kernel<TQ, SEL>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((d.nb + TQ - 1) / TQ, (unsigned)d.BH());
-  block_scores_kernel<TQ, SEL><<<grid, kThreads, smem, st>>>(qp, kp, vp, scale, P, vbar, d.nb, fs);
+  dim3 grid((d.nq + TQ - 1) / TQ, (unsigned)d.BH());
+  block_scores_kernel<TQ, SEL><<<grid, kThreads, smem, st>>>(qp, kp, vp, scale, P, vbar, d.nq, d.nk, fs);
   return cudaGetLastError();
 }
 
@@ -464,8 +473,8 @@ static cudaError_t scores_any(const Dims &d, const float *qp, const float *kp, c
                               cudaStream_t st) {
   // 16 rows per CTA while their logits fit comfortably in shared memory and the grid
   // still gives every SM two CTAs (296 on a 148-SM B200), else 8.
-  const long long ctas16 = (long long)((d.nb + 15) / 16) * d.BH();
-  if ((size_t)16 * d.nb * sizeof(float) <= 150 * 1024 && ctas16 >= 2 * 148)
+  const long long ctas16 = (long long)((d.nq + 15) / 16) * d.BH();
+  if ((size_t)16 * d.nk * sizeof(float) <= 150 * 1024 && ctas16 >= 2 * 148)
     return scores_tq<16, SEL>(d, qp, kp, vp, scale, P, vbar, fs, st);
   return scores_tq<8, SEL>(d, qp, kp, vp, scale, P, vbar, fs, st);
 }
@@ -491,26 +500,27 @@ cudaError_t launch_scores_select(const Dims &d, const ScoresSelectLaunch &a, cud
   return scores_any<true>(d, a.qp, a.kp, a.vp, a.scale, a.P, a.vbar, fs, st);
 }
 
+// workspace: w [BH, nq, 64] | a [BH, nq] | c [BH, nk], each 256-byte aligned
 size_t drift_workspace_bytes(const Dims &d) {
-  const size_t n = (size_t)d.BH() * d.nb;
+  const size_t nr = (size_t)d.BH() * d.nq, nc = (size_t)d.BH() * d.nk;
   auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
-  return up(n * kHeadDim * sizeof(float)) + up(n * sizeof(float)) * 2;
+  return up(nr * kHeadDim * sizeof(float)) + up(nr * sizeof(float)) + up(nc * sizeof(float));
 }
 
 cudaError_t launch_drift(const Dims &d, const float *P, const float *vp, const float *vbar,
                          const float *gram, float *s, void *ws, cudaStream_t st) {
-  const size_t n = (size_t)d.BH() * d.nb;
+  const size_t nr = (size_t)d.BH() * d.nq;
   auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
   char *base = static_cast<char *>(ws);
   float *w = reinterpret_cast<float *>(base);
-  float *a = reinterpret_cast<float *>(base + up(n * kHeadDim * sizeof(float)));
-  float *c = reinterpret_cast<float *>(base + up(n * kHeadDim * sizeof(float)) + up(n * sizeof(float)));
-  dim3 g1((d.nb + 31) / 32, (unsigned)d.BH(), 2);
-  drift_prep_kernel<<<g1, kThreads, 0, st>>>(vp, vbar, gram, w, a, c, d.H, d.nb);
+  float *a = reinterpret_cast<float *>(base + up(nr * kHeadDim * sizeof(float)));
+  float *c = reinterpret_cast<float *>(base + up(nr * kHeadDim * sizeof(float)) + up(nr * sizeof(float)));
+  dim3 g1((max(d.nq, d.nk) + 31) / 32, (unsigned)d.BH(), 2);
+  drift_prep_kernel<<<g1, kThreads, 0, st>>>(vp, vbar, gram, w, a, c, d.H, d.nq, d.nk);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  dim3 g2((d.nb + kDriftRows - 1) / kDriftRows, (unsigned)d.BH());
-  drift_kernel<<<g2, kThreads, 0, st>>>(P, vp, w, a, c, s, d.nb);
+  dim3 g2((d.nq + kDriftRows - 1) / kDriftRows, (unsigned)d.BH());
+  drift_kernel<<<g2, kThreads, 0, st>>>(P, vp, w, a, c, s, d.nq, d.nk);
   return cudaGetLastError();
 }
 

@@ -25,7 +25,7 @@ constexpr uint8_t F_TO_DROP = 4;  // chosen for drop this round
 constexpr uint8_t F_CAND = 5;     // candidate before the initial selection
 
 struct SelectParams {
-  int H, nb, method, rounds;
+  int H, nb, nq, method, rounds;  // nb: key blocks per row (nk), nq: query blocks
   int objective;  // ress_drift_objective
   float top_p;    // RESS_SELECT_CDF threshold
   float *drift;   // realized J per row, or null
@@ -144,7 +144,7 @@ __host__ __device__ __forceinline__ size_t select_warp_bytes(int nb, bool cdf = 
 
 __global__ void __launch_bounds__(512) select_kernel(const __grid_constant__ SelectParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  const int T = p.rows_per_cta, nb = p.nb;
+  const int T = p.rows_per_cta, nb = p.nb, nq = p.nq;  // nb = key blocks (nk)
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nthreads = blockDim.x;
   const bool drift = p.method == RESS_SELECT_DRIFT;
@@ -177,11 +177,11 @@ __global__ void __launch_bounds__(512) select_kernel(const __grid_constant__ Sel
   const long long bh = blockIdx.y;
   const int h = (int)(bh % p.H);
   const int i = blockIdx.x * T + warp;
-  const bool row_live = i < nb;
+  const bool row_live = i < nq;
   const bool dense = row_live && p.dense_q != nullptr && p.dense_q[i] != 0;
   const bool active = row_live && !dense;  // takes part in selection
-  const float *prow = p.P + ((size_t)bh * nb + (row_live ? i : 0)) * nb;
-  const float *srow = p.s ? p.s + ((size_t)bh * nb + (row_live ? i : 0)) * nb : nullptr;
+  const float *prow = p.P + ((size_t)bh * nq + (row_live ? i : 0)) * nb;
+  const float *srow = p.s ? p.s + ((size_t)bh * nq + (row_live ? i : 0)) * nb : nullptr;
   const float *vph = p.vp ? p.vp + (size_t)bh * nb * kHeadDim : nullptr;
 
   if (state) {
@@ -216,7 +216,7 @@ __global__ void __launch_bounds__(512) select_kernel(const __grid_constant__ Sel
                      [&](int j) { flags[j] = F_CAND; }, fixed, p.top_p, sorted);
       }
     } else if (p.method == RESS_SELECT_RANDOM) {
-      const uint64_t base = ((uint64_t)bh * nb + (uint64_t)i) * (uint64_t)nb;
+      const uint64_t base = ((uint64_t)bh * nq + (uint64_t)i) * (uint64_t)nb;
       warp_select<uint64_t>(nb, c, [&](int j) { return splitmix64_key(p.seed, base + (uint64_t)j + 1); },
                            is_cand, keep, hist, slot);
     } else {
@@ -241,7 +241,7 @@ __global__ void __launch_bounds__(512) select_kernel(const __grid_constant__ Sel
     const bool gather = active && (work || want_J);              // initial g and K
     float vb0 = 0.f, vb1 = 0.f;
     if (active) {
-      const float *vbr = p.vbar + ((size_t)bh * nb + i) * kHeadDim;
+      const float *vbr = p.vbar + ((size_t)bh * nq + i) * kHeadDim;
       vb0 = vbr[lane];
       vb1 = vbr[lane + 32];
     }
@@ -328,9 +328,9 @@ __global__ void __launch_bounds__(512) select_kernel(const __grid_constant__ Sel
         float *rgain = reinterpret_cast<float *>(rb + 1440);
         const uint8_t *rflags = rb + 1440 + (size_t)nb * 4;
         const int ri = blockIdx.x * T + rr;
-        const float *rp = p.P + ((size_t)bh * nb + (ri < nb ? ri : 0)) * nb;
-        const float *rsr = p.s + ((size_t)bh * nb + (ri < nb ? ri : 0)) * nb;
-        const bool rvalid = rlive && ri < nb;
+        const float *rp = p.P + ((size_t)bh * nq + (ri < nq ? ri : 0)) * nb;
+        const float *rsr = p.s + ((size_t)bh * nq + (ri < nq ? ri : 0)) * nb;
+        const bool rvalid = rlive && ri < nq;
         // P and s of this lane's blocks, fetched one tile ahead (up to 4 block groups
         // per warp: T >= 4 rows per CTA)
         float pn[4][2], sn[4][2];
@@ -426,13 +426,13 @@ __global__ void __launch_bounds__(512) select_kernel(const __grid_constant__ Sel
     // realized drift of the returned selection ([ReSS] §6.1): the tracked J after the
     // rounds, else the initial one; a dense query block drops nothing
     if (want_J && row_live && lane == 0)
-      p.drift[(size_t)bh * nb + i] = active ? (work ? bestJ : J) : 0.f;
+      p.drift[(size_t)bh * nq + i] = active ? (work ? bestJ : J) : 0.f;
   }
 
   // outputs: ascending kept list, count, optional mask
   if (row_live) {
-    int32_t *out = p.kv_idx + ((size_t)bh * nb + i) * nb;
-    uint8_t *mrow = p.mask ? p.mask + ((size_t)bh * nb + i) * nb : nullptr;
+    int32_t *out = p.kv_idx + ((size_t)bh * nq + i) * nb;
+    uint8_t *mrow = p.mask ? p.mask + ((size_t)bh * nq + i) * nb : nullptr;
     int total = 0;
     for (int base = 0; base < nb; base += 32) {
       const int j = base + lane;
@@ -442,7 +442,7 @@ __global__ void __launch_bounds__(512) select_kernel(const __grid_constant__ Sel
       if (mrow && j < nb) mrow[j] = k ? 1 : 0;
       total += __popc(bal);
     }
-    if (lane == 0) p.kv_cnt[(size_t)bh * nb + i] = total;
+    if (lane == 0) p.kv_cnt[(size_t)bh * nq + i] = total;
   }
 }
 
@@ -564,7 +564,8 @@ static size_t select_smem(int nb, int T, bool restore, bool state, bool cdf) {
 cudaError_t launch_select(const Dims &d, const SelectLaunch &a, cudaStream_t st) {
   SelectParams p{};
   p.H = d.H;
-  p.nb = d.nb;
+  p.nb = d.nk;
+  p.nq = d.nq;
   p.method = a.method;
   p.rounds = a.rounds;
   p.rho = a.rho;
@@ -592,31 +593,31 @@ cudaError_t launch_select(const Dims &d, const SelectLaunch &a, cudaStream_t st)
   // a grid that fills the GPU at small nb
   int T = restore ? 16 : 4;
   const bool cdf = a.method == RESS_SELECT_CDF;
-  while (T > 4 && select_smem(d.nb, T, restore, state, cdf) > 220 * 1024) T >>= 1;
+  while (T > 4 && select_smem(d.nk, T, restore, state, cdf) > 220 * 1024) T >>= 1;
   p.rows_per_cta = T;
-  const size_t smem = select_smem(d.nb, T, restore, state, cdf);
+  const size_t smem = select_smem(d.nk, T, restore, state, cdf);
   cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((d.nb + T - 1) / T, (unsigned)d.BH());
+  dim3 grid((d.nq + T - 1) / T, (unsigned)d.BH());
   select_kernel<<<grid, 32 * T, smem, st>>>(p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_schedule(const Dims &d, const int32_t *kv_cnt, int32_t *order, cudaStream_t st) {
-  const size_t par_smem = sizeof(int) * 33 * (size_t)(d.nb + 1);
+  const size_t par_smem = sizeof(int) * 33 * (size_t)(d.nk + 1);
   if (par_smem <= 200 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(schedule_kernel_par,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)par_smem);
     if (e != cudaSuccess) return e;
-    schedule_kernel_par<<<1, 1024, par_smem, st>>>(kv_cnt, order, d.BH() * d.nb, d.nb);
+    schedule_kernel_par<<<1, 1024, par_smem, st>>>(kv_cnt, order, d.BH() * d.nq, d.nk);
     return cudaGetLastError();
   }
-  const size_t smem = sizeof(int) * (d.nb + 1);
+  const size_t smem = sizeof(int) * (d.nk + 1);
   cudaError_t e = cudaFuncSetAttribute(schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  schedule_kernel<<<1, 1024, smem, st>>>(kv_cnt, order, d.BH() * d.nb, d.nb);
+  schedule_kernel<<<1, 1024, smem, st>>>(kv_cnt, order, d.BH() * d.nq, d.nk);
   return cudaGetLastError();
 }
 

@@ -12,7 +12,7 @@ using ress::Dims;
 
 namespace {
 
-constexpr int32_t kAbiVersion = 3;
+constexpr int32_t kAbiVersion = 4;
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -22,14 +22,20 @@ ress_status check_shape(const ress_shape *s, Dims *d, bool *empty) {
   if (s == nullptr) return RESS_ERR_INVALID_ARG;
   if (s->batch < 0 || s->seq_len < 0 || s->heads < 1) return RESS_ERR_INVALID_ARG;
   if (s->head_dim != ress::kHeadDim || s->block != ress::kBlock) return RESS_ERR_UNSUPPORTED;
+  if (s->key_block != 0 && s->key_block != ress::kBlock && s->key_block != ress::kBlock / 2)
+    return RESS_ERR_UNSUPPORTED;
   if (s->heads > ress::kMaxHeads) return RESS_ERR_UNSUPPORTED;
   d->B = s->batch;
   d->H = s->heads;
   d->N = s->seq_len;
-  d->nb = (s->seq_len + ress::kBlock - 1) / ress::kBlock;
-  if (d->nb > ress::kMaxBlocks) return RESS_ERR_UNSUPPORTED;
+  d->kb = s->key_block == 0 ? ress::kBlock : s->key_block;
+  d->nq = (s->seq_len + ress::kBlock - 1) / ress::kBlock;
+  d->nk = (s->seq_len + d->kb - 1) / d->kb;
+  d->nb = d->nq;
+  if (d->nk > ress::kMaxBlocks) return RESS_ERR_UNSUPPORTED;
   if (d->BH() > 65535) return RESS_ERR_UNSUPPORTED;  // grid.y limit of the block kernels
-  if (d->BH() * d->nb > 0x7fffffffll) return RESS_ERR_UNSUPPORTED;
+  if (d->BH() * d->nq * (long long)d->nk > 0x7fffffffffffll) return RESS_ERR_UNSUPPORTED;
+  if (d->BH() * d->nq > 0x7fffffffll) return RESS_ERR_UNSUPPORTED;
   *empty = (d->B == 0 || d->N == 0);
   return RESS_OK;
 }
@@ -149,7 +155,7 @@ ress_status ress_select_blocks(const ress_shape *shape, const ress_select_params
     return RESS_ERR_INVALID_ARG;
   if (m == RESS_SELECT_CDF && !(params->top_p > 0.f && params->top_p <= 1.f)) return RESS_ERR_INVALID_ARG;
   for (int h = 0; h < d.H; ++h)
-    if (params->budgets[h] < 0 || params->budgets[h] > d.nb) return RESS_ERR_INVALID_ARG;
+    if (params->budgets[h] < 0 || params->budgets[h] > d.nk) return RESS_ERR_INVALID_ARG;
   const int obj = params->objective;
   if (obj != RESS_DRIFT_MINIMISE && obj != RESS_DRIFT_MAXIMISE_SWAPS && obj != RESS_DRIFT_MAXIMISE_FULL)
     return RESS_ERR_INVALID_ARG;
@@ -209,7 +215,7 @@ ress_status ress_scores_select(const ress_shape *shape, const ress_select_params
   if (m == RESS_SELECT_CDF && !(params->top_p > 0.f && params->top_p <= 1.f)) return RESS_ERR_INVALID_ARG;
   if (params->objective != RESS_DRIFT_MINIMISE || params->drift != nullptr) return RESS_ERR_INVALID_ARG;
   for (int h = 0; h < d.H; ++h)
-    if (params->budgets[h] < 0 || params->budgets[h] > d.nb) return RESS_ERR_INVALID_ARG;
+    if (params->budgets[h] < 0 || params->budgets[h] > d.nk) return RESS_ERR_INVALID_ARG;
   if (!(scale > 0.f) || scale != scale) return RESS_ERR_INVALID_ARG;
   if (empty) return RESS_OK;
   if (!ptr_ok(q_pool) || !ptr_ok(k_pool) || !ptr_ok(kv_idx) || !ptr_ok(kv_cnt)) return RESS_ERR_INVALID_ARG;

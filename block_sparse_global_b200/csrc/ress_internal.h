@@ -10,8 +10,10 @@
 
 namespace ress {
 
+// nq query blocks of 128 tokens, nk key blocks of kb tokens (128, or 64 for the pages'
+// grid); nb == nq.
 struct Dims {
-  int B, H, N, nb;
+  int B, H, N, nb, nq, nk, kb;
   long long BH() const { return 1ll * B * H; }
 };
 

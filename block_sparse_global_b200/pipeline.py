@@ -18,26 +18,31 @@ from . import ress as R
 
 
 class SparseGlobalAttention:
-    def __init__(self, batch: int, heads: int, seq_len: int, device="cuda", with_mask: bool = False):
+    def __init__(self, batch: int, heads: int, seq_len: int, device="cuda", with_mask: bool = False,
+                 key_block: int = 128):
+        """key_block: tokens per key block, 128 (the query block's size) or 64 (ReSS
+        Supp. F).  Query blocks are always 128 tokens."""
         self.B, self.H, self.N = batch, heads, seq_len
-        self.nb = (seq_len + R.BLOCK - 1) // R.BLOCK
-        self.shape = R.make_shape(batch, heads, seq_len)
+        self.key_block = key_block
+        self.nq, self.nk = R.grid(seq_len, key_block)
+        self.nb = self.nq  # rows of the block map
+        self.shape = R.make_shape(batch, heads, seq_len, key_block=key_block)
         self.device = torch.device(device)
-        B, H, nb, N = batch, heads, self.nb, seq_len
+        B, H, nq, nk, N = batch, heads, self.nq, self.nk, seq_len
         f32 = dict(device=self.device, dtype=torch.float32)
         i32 = dict(device=self.device, dtype=torch.int32)
-        self.q_pool = torch.empty(B, H, nb, 64, **f32)
-        self.k_pool = torch.empty(B, H, nb, 64, **f32)
-        self.v_pool = torch.empty(B, H, nb, 64, **f32)
-        self.P = torch.empty(B, H, nb, nb, **f32)
-        self.v_bar = torch.empty(B, H, nb, 64, **f32)
-        self.s = torch.empty(B, H, nb, nb, **f32)
+        self.q_pool = torch.empty(B, H, nq, 64, **f32)
+        self.k_pool = torch.empty(B, H, nk, 64, **f32)
+        self.v_pool = torch.empty(B, H, nk, 64, **f32)
+        self.P = torch.empty(B, H, nq, nk, **f32)
+        self.v_bar = torch.empty(B, H, nq, 64, **f32)
+        self.s = torch.empty(B, H, nq, nk, **f32)
         self.workspace = torch.empty(max(R.ress_drift_workspace_bytes(self.shape), 16),
                                      device=self.device, dtype=torch.uint8)
-        self.kv_idx = torch.empty(B, H, nb, nb, **i32)
-        self.kv_cnt = torch.empty(B, H, nb, **i32)
-        self.order = torch.empty(B * H * nb, **i32)
-        self.mask = torch.empty(B, H, nb, nb, device=self.device, dtype=torch.uint8) if with_mask else None
+        self.kv_idx = torch.empty(B, H, nq, nk, **i32)
+        self.kv_cnt = torch.empty(B, H, nq, **i32)
+        self.order = torch.empty(B * H * nq, **i32)
+        self.mask = torch.empty(B, H, nq, nk, device=self.device, dtype=torch.uint8) if with_mask else None
         self.out = torch.empty(B, H, N, 64, device=self.device, dtype=torch.bfloat16)
         self.lse = torch.empty(B, H, N, **f32)
         self.dev_err = torch.zeros(4, **i32)
@@ -77,7 +82,7 @@ class SparseGlobalAttention:
                objective: int = R.DRIFT_MINIMISE, drift_out: Optional[torch.Tensor] = None,
                top_p: float = 1.0):
         """Block selection.  `objective` flips the sign of the drift objective (the
-        maximising controls, drift only); `drift_out` (fp32 [B,H,nb]) receives each row's
+        maximising controls, drift only); `drift_out` (fp32 [B,H,nq]) receives each row's
         realized drift J."""
         params = R.select_params(method, budgets, keep_k, dense_q, rounds, rho, eps, seed,
                                  objective, drift_out, top_p)
@@ -119,7 +124,8 @@ class SparseGlobalAttention:
         self._groups = []
         for g in range(groups):
             h0, h1 = bounds[g], bounds[g + 1]
-            sub = SparseGlobalAttention(1, h1 - h0, self.N, device=self.device)
+            sub = SparseGlobalAttention(1, h1 - h0, self.N, device=self.device,
+                                        key_block=self.key_block)
             sub.load_output_projection(w_o[:, 64 * h0:64 * h1])
             self._groups.append((h0, h1, sub))
         self._streams = [torch.cuda.Stream(self.device) for _ in range(3)]
@@ -177,13 +183,14 @@ class SparseGlobalAttention:
         return int(self.dev_err[0].item())
 
     def kept_lists(self):
-        """{(b,h,i): ascending kept key blocks} from the device kv list (host copy)."""
+        """{(b,h,i): ascending kept key blocks} from the device kv list (host copy); i runs
+        over the nq query blocks."""
         idx = self.kv_idx.cpu()
         cnt = self.kv_cnt.cpu()
         out = {}
         for b in range(self.B):
             for h in range(self.H):
-                for i in range(self.nb):
+                for i in range(self.nq):
                     c = int(cnt[b, h, i])
                     out[(b, h, i)] = idx[b, h, i, :c].tolist()
         return out

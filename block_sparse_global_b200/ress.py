@@ -33,7 +33,8 @@ class RessError(RuntimeError):
 
 class ress_shape(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("heads", ctypes.c_int32), ("seq_len", ctypes.c_int32),
-                ("head_dim", ctypes.c_int32), ("block", ctypes.c_int32)]
+                ("head_dim", ctypes.c_int32), ("block", ctypes.c_int32),
+                ("key_block", ctypes.c_int32)]
 
 
 class ress_select_params(ctypes.Structure):
@@ -111,8 +112,16 @@ def _stream(stream) -> Optional[int]:
 
 
 def make_shape(batch: int, heads: int, seq_len: int, head_dim: int = HEAD_DIM,
-               block: int = BLOCK) -> ress_shape:
-    return ress_shape(batch, heads, seq_len, head_dim, block)
+               block: int = BLOCK, key_block: int = 0) -> ress_shape:
+    """key_block 0 means key blocks of the query block's size (128); 64 is the grid of
+    ReSS Supp. F (128-token query blocks, 64-token key blocks)."""
+    return ress_shape(batch, heads, seq_len, head_dim, block, key_block)
+
+
+def grid(seq_len: int, key_block: int = 0):
+    """(nq, nk): query blocks of 128 tokens and key blocks of key_block tokens."""
+    kb = key_block or BLOCK
+    return (seq_len + BLOCK - 1) // BLOCK, (seq_len + kb - 1) // kb
 
 
 def _shape(shape) -> ress_shape:

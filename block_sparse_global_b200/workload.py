@@ -149,8 +149,8 @@ class Workload:
     k: torch.Tensor
     v: torch.Tensor
     w_o: torch.Tensor             # fp32 [d, H*64]: output projection, head h = columns 64h..64h+63
-    keep_k: torch.Tensor          # uint8 [nb]: always-kept key blocks (hold special tokens)
-    dense_q: torch.Tensor         # uint8 [nb]: query blocks computed densely
+    keep_k: torch.Tensor          # uint8 [nk]: always-kept key blocks (hold special tokens)
+    dense_q: torch.Tensor         # uint8 [nq]: query blocks computed densely
     budgets: list[int]            # per head, candidate blocks kept per row
     method: int
     rounds: int
@@ -159,6 +159,7 @@ class Workload:
     select_seed: int = 0
     sparsity: float = 0.0
     extras: dict = field(default_factory=dict)
+    key_block: int = BLOCK        # tokens per key block (query blocks are always BLOCK)
 
     @property
     def shape(self):
@@ -168,6 +169,14 @@ class Workload:
     @property
     def nb(self) -> int:
         return num_blocks(self.q.shape[2])
+
+    @property
+    def nq(self) -> int:
+        return num_blocks(self.q.shape[2])
+
+    @property
+    def nk(self) -> int:
+        return num_blocks(self.q.shape[2], self.key_block)
 
 
 def _vggt_qkv(case: Case, gen: torch.Generator, device) -> tuple:
@@ -206,10 +215,13 @@ def _vggt_qkv(case: Case, gen: torch.Generator, device) -> tuple:
 
 def make_workload(index: int, layer: int = 0, device="cpu", method: Optional[str] = None,
                   sparsity: Optional[float] = None, rounds: Optional[int] = None,
-                  heads: Optional[int] = None, views: Optional[int] = None) -> Workload:
+                  heads: Optional[int] = None, views: Optional[int] = None,
+                  key_block: int = BLOCK) -> Workload:
     """Build the seeded inputs of one synthetic case.  `method`, `sparsity`, `rounds`,
     `heads` and `views` override the case's own values (used by the sweep and by tests
-    that need a smaller VGGT-shaped layer)."""
+    that need a smaller VGGT-shaped layer).  `key_block` (128 or 64) sets the key-block
+    grid: keep_k and the budgets count key blocks of that size, dense_q query blocks of
+    128; Q, K, V and W_O do not depend on it."""
     case = CASES[index]
     if heads is not None or views is not None:
         hv = heads if heads is not None else case.heads
@@ -234,14 +246,16 @@ def make_workload(index: int, layer: int = 0, device="cpu", method: Optional[str
         n_special = case.views * VIEW_SPECIAL
     d_model = H * HEAD_DIM
     w_o = torch.randn(d_model, d_model, generator=gen, device=device) / math.sqrt(d_model)
-    nb = num_blocks(N)
-    tail = special_tail_blocks(N, n_special)
-    keep_k = torch.zeros(nb, dtype=torch.uint8, device=device)
-    dense_q = torch.zeros(nb, dtype=torch.uint8, device=device)
-    if tail:
-        keep_k[tail] = 1
-        dense_q[tail] = 1
-    n_cand = nb - len(tail)
+    nq, nk = num_blocks(N), num_blocks(N, key_block)
+    tail_q = special_tail_blocks(N, n_special)
+    tail_k = special_tail_blocks(N, n_special, key_block)
+    keep_k = torch.zeros(nk, dtype=torch.uint8, device=device)
+    dense_q = torch.zeros(nq, dtype=torch.uint8, device=device)
+    if tail_k:
+        keep_k[tail_k] = 1
+    if tail_q:
+        dense_q[tail_q] = 1
+    n_cand = nk - len(tail_k)
     s = case.sparsity if sparsity is None else sparsity
     c = uniform_budget(s, n_cand)
     budgets = [c] * H
@@ -259,4 +273,5 @@ def make_workload(index: int, layer: int = 0, device="cpu", method: Optional[str
                     q=q.to(bf).contiguous(), k=k.to(bf).contiguous(), v=v.to(bf).contiguous(),
                     w_o=w_o.float().contiguous(), keep_k=keep_k, dense_q=dense_q,
                     budgets=budgets, method=METHOD_NAMES[m], rounds=r,
-                    select_seed=seed * 7919 + 17, sparsity=s, extras=extras)
+                    select_seed=seed * 7919 + 17, sparsity=s, extras=extras,
+                    key_block=key_block)

@@ -27,20 +27,24 @@
  *   - Work is enqueued on `stream` and the call returns without synchronising.  Calls on
  *     one stream are ordered; calls on different streams may run concurrently as long
  *     as they do not write the same buffers.
- *   - Shapes: B = batch, H = heads, N = tokens, D = head_dim, b = block,
- *     nb = ceil(N / b) blocks (nq = nk = nb).  This version supports D = 64 and
- *     b = 128, 1 <= H <= 128 and nb <= 4096 (the paper's own per-row cap of 4096 key
- *     blocks, [ReSS] Supp. E).  B = 0 or N = 0 is an empty problem: the call returns
- *     RESS_OK and launches nothing.
- *   - Layouts are dense row-major: bf16 Q/K/V/out are [B, H, N, 64]; pooled tensors are
- *     fp32 [B, H, nb, 64]; block maps are fp32 [B, H, nb, nb]; the kept-block list is
- *     int32 kv_idx [B, H, nb, nb] (row = kept key blocks of one query block, ascending,
- *     entries past kv_cnt unspecified) with int32 kv_cnt [B, H, nb].
+ *   - Shapes: B = batch, H = heads, N = tokens, D = head_dim, b = query block,
+ *     b_k = key block (shape.key_block; 0 means b), nq = ceil(N / b) query blocks and
+ *     nk = ceil(N / b_k) key blocks.  This version supports D = 64, b = 128, b_k = 128
+ *     (nq = nk; written nb below where the two are the same) or b_k = 64 (the pages'
+ *     grid of 128-token query blocks and 64-token key blocks, [ReSS] Supp. F),
+ *     1 <= H <= 128 and nk <= 4096 (the paper's own per-row cap of 4096 key blocks,
+ *     [ReSS] Supp. E).  B = 0 or N = 0 is an empty problem: the call returns RESS_OK and
+ *     launches nothing.
+ *   - Layouts are dense row-major: bf16 Q/K/V/out are [B, H, N, 64]; pooled queries are
+ *     fp32 [B, H, nq, 64], pooled keys and values [B, H, nk, 64]; block maps are fp32
+ *     [B, H, nq, nk]; the kept-block list is int32 kv_idx [B, H, nq, nk] (row = kept key
+ *     blocks of one query block, ascending, entries past kv_cnt unspecified) with int32
+ *     kv_cnt [B, H, nq].  Per-query-block outputs (v_bar, drift) are [B, H, nq, ...].
  *   - Every pointer must be 16-byte aligned.
  *   - Errors: arguments are validated on the host before anything is launched; a bad
  *     argument returns RESS_ERR_INVALID_ARG or RESS_ERR_UNSUPPORTED and touches no
  *     memory.  A failed launch returns RESS_ERR_CUDA.  Problems found on the device (a
- *     kv_idx entry >= nb, kv_cnt > nb, an internal wait that timed out) are written to
+ *     kv_idx entry >= nk, kv_cnt > nk, an internal wait that timed out) are written to
  *     the optional int32 `dev_err` word with first-writer-wins (0 = none), the affected
  *     work is skipped, and the kernel never traps.  Read dev_err after synchronising.
  */
@@ -96,21 +100,22 @@ typedef struct {
   int32_t heads;    /* H, 1..128 */
   int32_t seq_len;  /* N >= 0 */
   int32_t head_dim; /* D, must be 64 */
-  int32_t block;    /* b, must be 128 */
+  int32_t block;    /* b, query block, must be 128 */
+  int32_t key_block; /* b_k, key block: 0 (= block), 128 or 64 */
 } ress_shape;
 
 typedef struct {
   int32_t method;           /* ress_method */
   const int32_t *budgets;   /* HOST [H]: c_h, candidate blocks kept per row of head h,
-                               0 <= c_h <= nb (else INVALID_ARG); a budget above the
+                               0 <= c_h <= nk (else INVALID_ARG); a budget above the
                                number of candidate (not always-kept) key blocks keeps
                                every candidate.  The paper keeps at least two key
                                blocks per row ([ReSS] Supp. F); that floor is the
                                caller's choice of budgets.                          */
-  const uint8_t *keep_k;    /* DEVICE [nb] or NULL: 1 = key block is always kept (holds
+  const uint8_t *keep_k;    /* DEVICE [nk] or NULL: 1 = key block is always kept (holds
                                special tokens, [ReSS] §3, §4.1); such blocks are never
                                candidates.  NULL = no always-kept block.            */
-  const uint8_t *dense_q;   /* DEVICE [nb] or NULL: 1 = this query block keeps every key
+  const uint8_t *dense_q;   /* DEVICE [nq] or NULL: 1 = this query block keeps every key
                                block (special query tokens are excluded from
                                sparsification, [ReSS] §3).  NULL = none.            */
   int32_t rounds;           /* R, restoration rounds for RESS_SELECT_DRIFT (0 = none);
@@ -118,21 +123,22 @@ typedef struct {
   float rho;                /* swap budget fraction of Eq. 17 (paper: 0.5), in (0, 1] */
   float eps;                /* guard of Eq. 7 (paper: 1e-4), > 0                      */
   uint64_t seed;            /* RESS_SELECT_RANDOM: key of pair (b,h,i,j) is output number
-                               ((b*H + h)*nb + i)*nb + j + 1 of a SplitMix64 generator
+                               ((b*H + h)*nq + i)*nk + j + 1 of a SplitMix64 generator
                                seeded with `seed` (Steele, Lea, Flood, OOPSLA 2014)   */
   int32_t objective;        /* ress_drift_objective; must be RESS_DRIFT_MINIMISE unless
                                method is RESS_SELECT_DRIFT (else INVALID_ARG)          */
   float top_p;              /* RESS_SELECT_CDF: mass threshold in (0, 1] (else INVALID_ARG);
                                ignored by the other methods                         */
-  float *drift;             /* DEVICE fp32 [B,H,nb] output or NULL: the realized drift J
+  float *drift;             /* DEVICE fp32 [B,H,nq] output or NULL: the realized drift J
                                of every row's final selection, Eq. 12 on its drop set
                                (Eq. 10) with K guarded by eps, for any method ([ReSS]
                                §6.1, Figs. 7 and 9); 0 for a dense_q row.  Needs
                                v_pool, v_bar and gram, and eps > 0.                 */
 } ress_select_params;
 
-/* Version of this ABI (incremented on any incompatible change): 3 (ress_select_params
- * gained `objective`, `top_p` and `drift`; RESS_SELECT_CDF). */
+/* Version of this ABI (incremented on any incompatible change): 4 (ress_shape gained
+ * `key_block`; ress_select_params gained `objective`, `top_p` and `drift`;
+ * RESS_SELECT_CDF). */
 int32_t ress_abi_version(void);
 
 /* Human-readable name of a status code (static string). */
@@ -171,10 +177,11 @@ ress_status ress_head_gram(const ress_shape *shape, int32_t d_model, const float
 
 /*
  * ress_pool_blocks -- block partition and mean pooling ([ReSS] §3 step (1); the pooled
- * values V_j of §4.1).  For every block j of tokens [128 j, min(N, 128 j + 128)):
+ * values V_j of §4.1).  For every block j of tokens [b j, min(N, b j + b)):
  * x_pool[b,h,j,:] = mean of those tokens' rows; the partial last block divides by its
- * true token count.  Reads bf16 q, k, v [B,H,N,64]; writes fp32 q_pool, k_pool,
- * v_pool [B,H,nb,64].  fp32 accumulation.
+ * true token count.  Queries are pooled over query blocks (q_pool [B,H,nq,64]), keys and
+ * values over key blocks (k_pool, v_pool [B,H,nk,64]).  Reads bf16 q, k, v [B,H,N,64].
+ * fp32 accumulation.
  */
 ress_status ress_pool_blocks(const ress_shape *shape, const void *q, const void *k,
                              const void *v, float *q_pool, float *k_pool, float *v_pool,
@@ -185,8 +192,8 @@ ress_status ress_pool_blocks(const ress_shape *shape, const void *q, const void 
  * ([ReSS] §3 step (1), §4.1 Eq. 1).
  *   P[b,h,i,j] = softmax over ALL key blocks j of (scale * q_pool_i . k_pool_j)
  *   v_bar[b,h,i,:] = sum_j P[b,h,i,j] v_pool[b,h,j,:]
- * scale: logit scale, normally 1/sqrt(64).  Outputs fp32 P [B,H,nb,nb] and
- * v_bar [B,H,nb,64].
+ * scale: logit scale, normally 1/sqrt(64).  Outputs fp32 P [B,H,nq,nk] and
+ * v_bar [B,H,nq,64].
  */
 ress_status ress_block_scores(const ress_shape *shape, const float *q_pool,
                               const float *k_pool, const float *v_pool, float scale,
@@ -205,7 +212,7 @@ size_t ress_drift_workspace_bytes(const ress_shape *shape);
  *   workspace  DEVICE scratch of at least ress_drift_workspace_bytes(shape) bytes,
  *              owned by the caller, 16-byte aligned; its contents are overwritten and
  *              are meaningless after the call.
- * Output fp32 s [B,H,nb,nb].
+ * Output fp32 s [B,H,nq,nk].
  */
 ress_status ress_drift_scores(const ress_shape *shape, const float *P, const float *v_pool,
                               const float *v_bar, const float *gram, float *s,
@@ -260,12 +267,12 @@ ress_status ress_drift_scores_static(const ress_shape *shape, const float *P,
  *            (and, for MAXIMISE_FULL, in the initial selection); the largest J seen is
  *            then returned.
  * Every top-k orders by (score descending, block index ascending).
- *   P       fp32 [B,H,nb,nb] (ress_block_scores).
- *   s       fp32 [B,H,nb,nb] (ress_drift_scores); required for DRIFT, else may be NULL.
+ *   P       fp32 [B,H,nq,nk] (ress_block_scores).
+ *   s       fp32 [B,H,nq,nk] (ress_drift_scores); required for DRIFT, else may be NULL.
  *   v_pool, v_bar, gram: required for DRIFT with rounds > 0 and whenever params->drift
  *           is set, else may be NULL.
- *   kv_idx  int32 [B,H,nb,nb] output; kv_cnt int32 [B,H,nb] output.
- *   mask    uint8 [B,H,nb,nb] output (1 = kept) or NULL.
+ *   kv_idx  int32 [B,H,nq,nk] output; kv_cnt int32 [B,H,nq] output.
+ *   mask    uint8 [B,H,nq,nk] output (1 = kept) or NULL.
  *   dev_err int32 device word or NULL.
  */
 ress_status ress_select_blocks(const ress_shape *shape, const ress_select_params *params,
@@ -283,9 +290,10 @@ ress_status ress_select_blocks(const ress_shape *shape, const ress_select_params
  *   params   as for ress_select_blocks; method must be MASS, CDF or RANDOM (else
  *            UNSUPPORTED: drift selection needs the drift score and restoration of
  *            its own calls), objective MINIMISE and drift NULL (else INVALID_ARG).
- *   q_pool, k_pool  fp32 [B,H,nb,64] (ress_pool_blocks); v_pool needed only with v_bar.
- *   P        fp32 [B,H,nb,nb] output or NULL (not written).
- *   v_bar    fp32 [B,H,nb,64] output or NULL (Eq. 1 output not computed).
+ *   q_pool [B,H,nq,64], k_pool [B,H,nk,64] fp32 (ress_pool_blocks); v_pool needed only
+ *            with v_bar.
+ *   P        fp32 [B,H,nq,nk] output or NULL (not written).
+ *   v_bar    fp32 [B,H,nq,64] output or NULL (Eq. 1 output not computed).
  *   kv_idx, kv_cnt, mask, dev_err: as for ress_select_blocks.
  */
 ress_status ress_scores_select(const ress_shape *shape, const ress_select_params *params,
@@ -296,11 +304,11 @@ ress_status ress_scores_select(const ress_shape *shape, const ress_select_params
 
 /*
  * ress_attn_schedule -- launch order for ress_block_sparse_attn: a permutation of the
- * B*H*nb (batch, head, query block) work items sorted by kv_cnt descending, ties in
- * ascending item order (item = (b*H + h)*nb + i).  Running the longest rows first keeps
+ * B*H*nq (batch, head, query block) work items sorted by kv_cnt descending, ties in
+ * ascending item order (item = (b*H + h)*nq + i).  Running the longest rows first keeps
  * rows that keep every block (dense query blocks) off the tail of the launch.
- *   kv_cnt     int32 [B,H,nb];  work_order int32 [B*H*nb] output.
- * Deterministic.  kv_cnt values outside [0, nb] are clamped for ordering only.
+ *   kv_cnt     int32 [B,H,nq];  work_order int32 [B*H*nq] output.
+ * Deterministic.  kv_cnt values outside [0, nk] are clamped for ordering only.
  */
 ress_status ress_attn_schedule(const ress_shape *shape, const int32_t *kv_cnt,
                                int32_t *work_order, ress_stream_t stream);
@@ -314,10 +322,10 @@ ress_status ress_attn_schedule(const ress_shape *shape, const int32_t *kv_cnt,
  * and lse[b,h,t] = ln sum_u exp(scale * q_t . k_u).  A row with kv_cnt = 0 gets zero
  * output and lse = -inf.  kv_idx rows need not be sorted.
  *   q, k, v     bf16 [B,H,N,64];  out bf16 [B,H,N,64];  lse fp32 [B,H,N] or NULL.
- *   work_order  int32 [B*H*nb] permutation from ress_attn_schedule, or NULL for the
+ *   work_order  int32 [B*H*nq] permutation from ress_attn_schedule, or NULL for the
  *               natural order.  Outputs do not depend on it.
- *   dev_err     int32 device word or NULL: an entry of kv_idx outside [0, nb) or a
- *               kv_cnt outside [0, nb] sets RESS_ERR_DEVICE_BOUNDS and that row is
+ *   dev_err     int32 device word or NULL: an entry of kv_idx outside [0, nk) or a
+ *               kv_cnt outside [0, nk] sets RESS_ERR_DEVICE_BOUNDS and that row is
  *               left unwritten.
  * Implementation: bf16 tensor-core tiles (tcgen05, accumulators in tensor memory) fed
  * by TMA, fp32 online softmax.

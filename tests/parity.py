@@ -40,7 +40,8 @@ def run_gpu(wl, method=None, rounds=None, with_mask=True, seed=None):
         rounds = 0
     q, k, v = wl.q.to(dev), wl.k.to(dev), wl.v.to(dev)
     b, h, n, _ = q.shape
-    layer = SparseGlobalAttention(b, h, n, device=dev, with_mask=with_mask)
+    layer = SparseGlobalAttention(b, h, n, device=dev, with_mask=with_mask,
+                                  key_block=wl.key_block)
     layer.load_output_projection(wl.w_o.to(dev))
     layer.forward(q, k, v, method, wl.budgets, wl.keep_k.to(dev), wl.dense_q.to(dev), rounds,
                   wl.rho, wl.eps, wl.select_seed if seed is None else seed)
@@ -63,12 +64,14 @@ class OracleLayer:
         self.v = O.to_numpy_f32(wl.v)
         self.B, self.H, self.N, _ = self.q.shape
         self.scale = 1.0 / math.sqrt(64)
+        self.key_block = wl.key_block
         self.qp = O.pool_blocks(self.q)
-        self.kp = O.pool_blocks(self.k)
-        self.vp = O.pool_blocks(self.v)
+        self.kp = O.pool_blocks(self.k, wl.key_block)
+        self.vp = O.pool_blocks(self.v, wl.key_block)
         self.P, self.vbar = O.block_scores(self.qp, self.kp, self.vp, self.scale)
         self.gram = O.head_gram(O.to_numpy_f32(wl.w_o), self.H)
-        self.nb = self.P.shape[-1]
+        self.nq, self.nk = self.P.shape[-2:]
+        self.nb = self.nk  # key blocks: the width of a kept-block mask
         self.keep_k = wl.keep_k.cpu().numpy()
         self.dense_q = wl.dense_q.cpu().numpy()
         self.wl = wl
@@ -96,7 +99,8 @@ class OracleLayer:
                                top_p=top_p)
 
     def attention(self, kept, rows):
-        return O.block_sparse_attn(self.q, self.k, self.v, kept, self.scale, rows=rows)
+        return O.block_sparse_attn(self.q, self.k, self.v, kept, self.scale, rows=rows,
+                                   key_block=self.key_block)
 
 
 def close(got, want, rtol, atol, what):

@@ -39,7 +39,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert R.ress_abi_version() == 3
+    assert R.ress_abi_version() == 4
     assert R.ress_status_string(0) == "RESS_OK"
     assert R.ress_status_string(5) == "RESS_ERR_DEVICE_TIMEOUT"
     assert R.ress_status_string(99) == "RESS_ERR_UNKNOWN"
@@ -58,6 +58,18 @@ def test_shape_validation(lib):
     assert _pool(lib, ctypes.byref(R.make_shape(1, 4, 4096 * 128 + 1)), ptrs) == UNSUPPORTED
     assert _pool(lib, ctypes.byref(R.make_shape(-1, 4, 1024)), ptrs) == INVALID
     assert _pool(lib, ctypes.byref(R.make_shape(1, 0, 1024)), ptrs) == INVALID
+    # key blocks: 0 (= the query block), 128 or 64 tokens; at most 4096 key blocks
+    for kb in (32, 96, 256, -64, 1):
+        assert _pool(lib, ctypes.byref(R.make_shape(1, 4, 1024, key_block=kb)), ptrs) == UNSUPPORTED
+    assert _pool(lib, ctypes.byref(R.make_shape(1, 4, 4096 * 64 + 1, key_block=64)),
+                 ptrs) == UNSUPPORTED
+
+
+def test_key_block_grid_sizes():
+    assert R.grid(1024) == (8, 8) and R.grid(1024, 128) == (8, 8)
+    assert R.grid(1024, 64) == (8, 16)
+    assert R.grid(4122, 64) == (33, 65)     # 3 VGGT views: ragged last blocks of 26 tokens
+    assert R.grid(1, 64) == (1, 1) and R.grid(0, 64) == (0, 0)
 
 
 def test_empty_problem_is_ok_without_launch(lib):
@@ -91,6 +103,10 @@ def test_select_parameter_validation(lib):
         return lib.ress_select_blocks(shape, ctypes.byref(p), *args)
 
     assert call(1, [4, 9]) == INVALID             # budget > nb
+    # with 64-token key blocks the same sequence has 16 key blocks: budgets count those
+    shape64 = ctypes.byref(R.make_shape(1, 2, 1024, key_block=64))
+    p, keep = R.select_params(1, [4, 17], rounds=2)
+    assert lib.ress_select_blocks(shape64, ctypes.byref(p), *args) == INVALID
     assert call(1, [4, -1]) == INVALID
     assert call(7, [4, 4]) == INVALID             # unknown method
     assert call(1, [4, 4], rounds=65) == INVALID

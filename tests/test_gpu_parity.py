@@ -253,22 +253,22 @@ def test_keep_all_is_dense_attention():
     assert err <= 2e-2 and rel <= 1e-2, (err, rel)
 
 
-def _manual_attn(N, lists, B=1, H=2, seed=0):
+def _manual_attn(N, lists, B=1, H=2, seed=0, key_block=128):
     ensure_built()
     g = torch.Generator(device="cuda").manual_seed(seed)
     q, k, v = (torch.randn(B, H, N, 64, device="cuda", generator=g).to(torch.bfloat16)
                for _ in range(3))
-    nb = (N + 127) // 128
-    kv_idx = torch.zeros(B, H, nb, nb, dtype=torch.int32)
-    kv_cnt = torch.zeros(B, H, nb, dtype=torch.int32)
+    nq, nk = R.grid(N, key_block)
+    kv_idx = torch.zeros(B, H, nq, nk, dtype=torch.int32)
+    kv_cnt = torch.zeros(B, H, nq, dtype=torch.int32)
     for (b, h, i), lst in lists.items():
         kv_cnt[b, h, i] = len(lst)
         kv_idx[b, h, i, :len(lst)] = torch.tensor(lst, dtype=torch.int32)
     out = torch.full((B, H, N, 64), 7.0, device="cuda", dtype=torch.bfloat16)
     lse = torch.empty(B, H, N, device="cuda")
     err = torch.zeros(1, device="cuda", dtype=torch.int32)
-    R.ress_block_sparse_attn(R.make_shape(B, H, N), q, k, v, kv_idx.cuda(), kv_cnt.cuda(), None,
-                             0.125, out, lse, err)
+    R.ress_block_sparse_attn(R.make_shape(B, H, N, key_block=key_block), q, k, v, kv_idx.cuda(),
+                             kv_cnt.cuda(), None, 0.125, out, lse, err)
     torch.cuda.synchronize()
     return q, k, v, out, lse, int(err.item())
 
@@ -449,3 +449,119 @@ def test_wide_logit_range_and_rescaling():
     assert (out.float() - ref).abs().max().item() <= 2e-2
     assert ((out.float() - ref).norm() / ref.norm()).item() <= 1e-2
     assert ((lse - lref).abs() <= 1e-3 + 1e-4 * lref.abs()).all()
+
+
+# ------------------------------------------- key blocks of 64 tokens (ReSS Supp. F grid)
+def test_key_block_64_edge_rows_odd_even_ragged_unsorted():
+    """Query blocks of 128 against key blocks of 64: N = 300 gives 3 query blocks and 5
+    key blocks, the last 44 tokens.  Rows with odd counts (the last tile's second half
+    empty), even counts, the ragged block in either half, unsorted lists, one block, the
+    ragged block alone and an empty row; oracle per query block."""
+    N = 300
+    lists = {(0, 0, 0): [4, 0, 2], (0, 0, 1): [], (0, 0, 2): [4], (0, 1, 0): [0, 1, 2, 3, 4],
+             (0, 1, 1): [1, 4], (0, 1, 2): [3, 1, 0, 2], (1, 0, 0): [2], (1, 0, 1): [4, 3],
+             (1, 0, 2): [0, 1, 2, 3], (1, 1, 0): [1, 0], (1, 1, 1): [0, 2, 4, 1, 3],
+             (1, 1, 2): [3]}
+    q, k, v, out, lse, err = _manual_attn(N, lists, B=2, key_block=64)
+    assert err == 0
+    qn, kn, vn = (O.to_numpy_f32(t) for t in (q, k, v))
+    for (b, h, i), lst in lists.items():
+        o_ref, l_ref = O.attention_qblock(qn, kn, vn, b, h, i, sorted(lst), 0.125, key_block=64)
+        r0 = i * 128
+        o = out[b, h, r0:r0 + o_ref.shape[0]].float().cpu().numpy()
+        assert np.abs(o - o_ref).max() <= 2e-2, (b, h, i, lst)
+        if lst:
+            close(lse[b, h, r0:r0 + o_ref.shape[0]].cpu(), l_ref, 1e-4, 1e-3, f"lse{(b, h, i)}")
+        else:
+            assert np.all(o == 0) and torch.isinf(lse[b, h, r0:r0 + o_ref.shape[0]]).all()
+
+
+def test_key_block_64_out_of_range_index_sets_device_error():
+    # 256 tokens: 4 key blocks of 64; index 4 is out of range and its row is skipped
+    lists = {(0, 0, 0): [0, 4], (0, 0, 1): [3], (0, 1, 0): [0], (0, 1, 1): [2, 1]}
+    q, k, v, out, lse, err = _manual_attn(256, lists, key_block=64)
+    assert err == 4   # RESS_ERR_DEVICE_BOUNDS
+    assert torch.all(out[0, 0, :128].float() == 7.0)       # the bad row is left unwritten
+    qn, kn, vn = (O.to_numpy_f32(t) for t in (q, k, v))
+    for r in ((0, 0, 1), (0, 1, 0), (0, 1, 1)):
+        o_ref, _ = O.attention_qblock(qn, kn, vn, *r, sorted(lists[r]), 0.125, key_block=64)
+        o = out[r[0], r[1], r[2] * 128:r[2] * 128 + 128].float().cpu().numpy()
+        assert np.abs(o - o_ref).max() <= 2e-2
+
+
+@pytest.mark.parametrize("method", ["mass", "drift", "random"])
+@pytest.mark.parametrize("sparsity", [0.6, 0.61])
+def test_key_block_64_small_layer_every_row(method, sparsity):
+    """The whole path on the 128 x 64 grid: 3 views, N = 4122 -> 33 query blocks and 65
+    key blocks, both ragged (58 and 26 tokens); the 15 special tokens sit in key block 64
+    (always kept) and query block 32 (dense).  Sparsity 0.6 keeps 26 candidates + 1 (an
+    odd count: the last score tile is half empty), 0.61 keeps 25 + 1 (even)."""
+    wl = W.make_workload(2, heads=2, views=3, method=method, sparsity=sparsity, rounds=4,
+                         key_block=64)
+    assert (wl.nq, wl.nk) == (33, 65)
+    assert wl.keep_k.nonzero().flatten().tolist() == [64]
+    assert wl.dense_q.nonzero().flatten().tolist() == [32]
+    rows = _all_rows(1, 2, wl.nq)
+    layer, orc, stats = _full_check(wl, METHODS[method], rows, rows, rounds=4)
+    kept = layer.kept_lists()
+    want = wl.budgets[0] + 1
+    assert want % 2 == (1 if sparsity == 0.6 else 0)
+    for (b, h, i), lst in kept.items():
+        assert 64 in lst
+        assert lst == list(range(65)) if i == 32 else len(lst) == want
+
+
+def test_key_block_64_vggt_8view_mass50_sampled():
+    """The 8-view layer (N = 10992: 86 query blocks, 172 key blocks) on the 128 x 64 grid:
+    block tensors everywhere, selection on every row, attention on sampled rows."""
+    wl = W.make_workload(2, key_block=64)
+    assert (wl.nq, wl.nk) == (86, 172)
+    rows = _all_rows(1, 16, wl.nq)
+    attn_rows = sample_rows(1, 16, wl.nq, 32, seed=7,
+                            always=[(0, 0, wl.nq - 1), (0, 15, wl.nq - 2), (0, 3, 0)])
+    layer, orc, stats = _full_check(wl, O.MASS, rows, attn_rows)
+    cnt = layer.kv_cnt.cpu()
+    assert int(cnt[0, 0, 0]) == wl.budgets[0] + int(wl.keep_k.sum())
+    assert int(cnt[0, 3, wl.nq - 1]) == wl.nk
+
+
+def test_key_block_64_vggt_32view_drift75_sampled():
+    wl = W.make_workload(3, key_block=64)
+    rows = sample_rows(1, 16, wl.nq, 48, seed=8, always=[(0, 0, wl.nq - 1), (0, 7, 0)])
+    attn_rows = sample_rows(1, 16, wl.nq, 12, seed=9, always=[(0, 5, wl.nq - 2)])
+    _full_check(wl, O.DRIFT, rows, attn_rows)
+
+
+@pytest.mark.parametrize("top_p", [0.5, 0.9])
+def test_key_block_64_cdf_on_oracle_scores(top_p):
+    wl = W.make_workload(2, heads=4, views=6, method="mass", sparsity=0.5, key_block=64)
+    ensure_built()
+    orc = OracleLayer(wl)
+    rows = _all_rows(1, 4, orc.nq)
+    dev = torch.device("cuda")
+    layer = SparseGlobalAttention(1, 4, wl.q.shape[2], device=dev, with_mask=True, key_block=64)
+    layer.P.copy_(torch.from_numpy(orc.P))
+    layer.select(O.CDF, wl.budgets, wl.keep_k.to(dev), wl.dense_q.to(dev), top_p=top_p)
+    torch.cuda.synchronize()
+    sel = orc.select(rows, O.CDF, 0, 0, top_p=top_p)
+    compare_masks(layer.kept_lists(), sel, orc.nk, f"cdf64/{top_p}")
+    fz = SparseGlobalAttention(1, 4, wl.q.shape[2], device=dev, with_mask=True, key_block=64)
+    fz.pool(wl.q.to(dev), wl.k.to(dev), wl.v.to(dev))
+    fz.scores_select(O.CDF, wl.budgets, wl.keep_k.to(dev), wl.dense_q.to(dev), top_p=top_p)
+    ref = SparseGlobalAttention(1, 4, wl.q.shape[2], device=dev, with_mask=True, key_block=64)
+    ref.scores(wl.q.to(dev), wl.k.to(dev), wl.v.to(dev))
+    ref.select(O.CDF, wl.budgets, wl.keep_k.to(dev), wl.dense_q.to(dev), top_p=top_p)
+    torch.cuda.synchronize()
+    # entries past kv_cnt are unspecified: compare the kept lists
+    assert torch.equal(fz.kv_cnt, ref.kv_cnt) and fz.kept_lists() == ref.kept_lists()
+
+
+def test_key_block_64_keep_all_is_dense_attention():
+    wl = W.make_workload(2, heads=4, views=4, method="mass", sparsity=0.0, key_block=64)
+    layer = run_gpu(wl)
+    assert int(layer.kv_cnt.min()) == wl.nk
+    q, k, v = (t.cuda().float() for t in (wl.q, wl.k, wl.v))
+    ref = torch.nn.functional.scaled_dot_product_attention(q, k, v, scale=0.125)
+    err = (layer.out.float() - ref).abs().max().item()
+    rel = ((layer.out.float() - ref).norm() / ref.norm()).item()
+    assert err <= 2e-2 and rel <= 1e-2, (err, rel)
