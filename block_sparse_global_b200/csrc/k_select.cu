@@ -316,87 +316,108 @@ __global__ void __launch_bounds__(512) select_kernel(const __grid_constant__ Sel
       }
       __syncwarp();
       // Gains of every candidate from the start-of-round state (Eqs. 14-16), computed by
-      // the whole CTA: a 64-block tile is 16 groups of four blocks; warp w takes groups
-      // w, w + T, ... and lane = (row lane & 15, block pair lane >> 4), so a tile row read
-      // from shared memory serves every row of the CTA at once.
+      // the whole CTA against 64-block tiles of the head's pooled values.  The d_j^T M g
+      // inner products of a tile form a (rows x 64 blocks) product over 64 dimensions;
+      // thread t takes a 4-row x 4-block micro-tile (row group rg, block group kg) over 8
+      // of the dimensions (slice ds: 4ds..4ds+3 and 32+4ds..32+4ds+3).  Its rows' M g
+      // slices stay in registers for the whole pass, so a tile costs each thread eight
+      // 16-byte shared-memory reads for 128 FMAs.  The 8 slices of a micro-tile sit on 8
+      // consecutive lanes; a transposing butterfly (xor 4, 2, 1) sums them and leaves lane
+      // ds with the products of row ds/2 and blocks 2(ds%2), 2(ds%2)+1, whose gains it
+      // writes.
       {
-        const int rr = lane & 15, kp = lane >> 4;
-        const bool rlive = rr < T;
-        unsigned char *rb = wbase + wbytes * (rlive ? rr : 0);
-        const float *rh = reinterpret_cast<const float *>(rb + 1152);
-        const float *rs = reinterpret_cast<const float *>(rb + 1408);
-        float *rgain = reinterpret_cast<float *>(rb + 1440);
-        const uint8_t *rflags = rb + 1440 + (size_t)nb * 4;
-        const int ri = blockIdx.x * T + rr;
-        const float *rp = p.P + ((size_t)bh * nq + (ri < nq ? ri : 0)) * nb;
-        const float *rsr = p.s + ((size_t)bh * nq + (ri < nq ? ri : 0)) * nb;
-        const bool rvalid = rlive && ri < nq;
-        // P and s of this lane's blocks, fetched one tile ahead (up to 4 block groups
-        // per warp: T >= 4 rows per CTA)
-        float pn[4][2], sn[4][2];
+        const int ds = threadIdx.x & 7, mt = threadIdx.x >> 3;
+        const int ngr = T >> 2;  // row groups of four (T = 4, 8 or 16)
+        const int rg = mt % ngr, kg = mt / ngr;
+        __syncthreads();  // every row's M g, scalars and flags of this round are written
+        float4 hv[4][2];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const unsigned char *rb = wbase + wbytes * (rg * 4 + r);
+          const bool live = reinterpret_cast<const int *>(rb + 1408)[4] == 1;
+          const float4 *hh = reinterpret_cast<const float4 *>(rb + 1152);
+          const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+          hv[r][0] = live ? hh[ds] : z;
+          hv[r][1] = live ? hh[8 + ds] : z;
+        }
+        // the (row, block) pairs whose gains this lane writes
+        const int re = rg * 4 + (ds >> 1);
+        unsigned char *eb = wbase + wbytes * re;
+        const float *es = reinterpret_cast<const float *>(eb + 1408);
+        float *egain = reinterpret_cast<float *>(eb + 1440);
+        const uint8_t *eflags = eb + 1440 + (size_t)nb * 4;
+        const int ei = blockIdx.x * T + re;
+        const bool ework = ei < nq && reinterpret_cast<const int *>(es)[4] == 1;
+        const float *ep = p.P + ((size_t)bh * nq + (ework ? ei : 0)) * nb;
+        const float *esr = p.s + ((size_t)bh * nq + (ework ? ei : 0)) * nb;
+        const float vh = es[0], base = es[1], G = es[2], Kr = es[3];
+        const int jq = kg * 4 + 2 * (ds & 1);  // first of the lane's two blocks in a tile
+        // P and s of this lane's two blocks, fetched one tile ahead
+        float pn[2], sn[2];
         auto fetch = [&](int tt) {
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            const int kg = warp + g * T;
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              const int j = tt * kTileKeys + 4 * kg + 2 * kp + q;
-              const bool ok = rvalid && kg < 16 && j < nb;
-              pn[g][q] = ok ? rp[j] : 0.f;
-              sn[g][q] = ok ? rsr[j] : 0.f;
-            }
+          for (int q = 0; q < 2; ++q) {
+            const int j = tt * kTileKeys + jq + q;
+            const bool ok = ework && j < nb;
+            pn[q] = ok ? ep[j] : 0.f;
+            sn[q] = ok ? esr[j] : 0.f;
           }
         };
         fetch(0);
+        const bool b2 = ds & 4, b1 = ds & 2, b0 = ds & 1;
         tile_stream_n<kSelStages>(tiles, vph, nb, [&](int tt, const float *tile) {
-          float pc[4][2], sc[4][2];
-#pragma unroll
-          for (int g = 0; g < 4; ++g)
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              pc[g][q] = pn[g][q];
-              sc[g][q] = sn[g][q];
-            }
+          const float pc[2] = {pn[0], pn[1]}, sc[2] = {sn[0], sn[1]};
           fetch(tt + 1);
-          // the rows' flags and scalars are read only here, after the stream's barrier
-          // has made every warp's writes of this round visible
-          if (!(rlive && reinterpret_cast<const int *>(rs)[4] == 1)) return;
-          const float vh = rs[0], base = rs[1], G = rs[2], Kr = rs[3];
-          const float4 *hh = reinterpret_cast<const float4 *>(rh);
+          float acc[16];
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            const int kg = warp + g * T;
-            if (kg >= 16) break;
-            const int kw = 4 * kg + 2 * kp;  // this lane's two blocks within the tile
-            const int j0 = tt * kTileKeys + kw;
-            const float4 *v0 = reinterpret_cast<const float4 *>(tile + kw * kTilePad);
-            const float4 *v1 = reinterpret_cast<const float4 *>(tile + (kw + 1) * kTilePad);
-            float d0 = 0.f, d1 = 0.f;
+          for (int kk = 0; kk < 4; ++kk) {
+            const float4 *vk = reinterpret_cast<const float4 *>(tile + (kg * 4 + kk) * kTilePad);
+            const float4 a = vk[ds], b = vk[8 + ds];
 #pragma unroll
-            for (int d = 0; d < 16; ++d) {
-              const float4 x = hh[d], y0 = v0[d], y1 = v1[d];
-              d0 = fmaf(y0.x, x.x, d0); d0 = fmaf(y0.y, x.y, d0); d0 = fmaf(y0.z, x.z, d0); d0 = fmaf(y0.w, x.w, d0);
-              d1 = fmaf(y1.x, x.x, d1); d1 = fmaf(y1.y, x.y, d1); d1 = fmaf(y1.z, x.z, d1); d1 = fmaf(y1.w, x.w, d1);
+            for (int r = 0; r < 4; ++r) {
+              const float4 x = hv[r][0], y = hv[r][1];
+              float d = a.x * x.x;
+              d = fmaf(a.y, x.y, d); d = fmaf(a.z, x.z, d); d = fmaf(a.w, x.w, d);
+              d = fmaf(b.x, y.x, d); d = fmaf(b.y, y.y, d); d = fmaf(b.z, y.z, d); d = fmaf(b.w, y.w, d);
+              acc[r * 4 + kk] = d;
             }
+          }
+          // butterfly: after the xor-4 / xor-2 / xor-1 steps lane ds holds the sums of
+          // products 2ds and 2ds + 1 (product index = 4 * row + block within the tile)
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              const int j = j0 + q;
-              if (j >= nb) continue;
-              const uint8_t f = rflags[j];
-              if (f != F_KEPT && f != F_DROP) continue;
-              const float pj = pc[g][q], sj = sc[g][q];
-              const float t = __fmul_rn(pj, __fsub_rn(vh, q == 0 ? d0 : d1));  // d_j^T M g
-              const float s2 = __fmul_rn(sj, sj);
-              float dG, Kn;
-              if (f == F_DROP) {  // restore j
-                dG = __fadd_rn(__fmul_rn(-2.f, t), s2);
-                Kn = fmaxf(__fadd_rn(Kr, pj), p.eps);
-              } else {            // drop j
-                dG = __fadd_rn(__fmul_rn(2.f, t), s2);
-                Kn = fmaxf(__fsub_rn(Kr, pj), p.eps);
-              }
-              rgain[j] = __fsub_rn(base, __fdiv_rn(__fadd_rn(G, dG), __fmul_rn(Kn, Kn)));
+          for (int i = 0; i < 8; ++i) {
+            const float send = b2 ? acc[i] : acc[8 + i], keep = b2 ? acc[8 + i] : acc[i];
+            acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+          }
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float send = b1 ? acc[i] : acc[4 + i], keep = b1 ? acc[4 + i] : acc[i];
+            acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+          }
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const float send = b0 ? acc[i] : acc[2 + i], keep = b0 ? acc[2 + i] : acc[i];
+            acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+          }
+          if (!ework) return;
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const int j = tt * kTileKeys + jq + q;
+            if (j >= nb) continue;
+            const uint8_t f = eflags[j];
+            if (f != F_KEPT && f != F_DROP) continue;
+            const float pj = pc[q], sj = sc[q];
+            const float t = __fmul_rn(pj, __fsub_rn(vh, acc[q]));  // d_j^T M g
+            const float s2 = __fmul_rn(sj, sj);
+            float dG, Kn;
+            if (f == F_DROP) {  // restore j
+              dG = __fadd_rn(__fmul_rn(-2.f, t), s2);
+              Kn = fmaxf(__fadd_rn(Kr, pj), p.eps);
+            } else {            // drop j
+              dG = __fadd_rn(__fmul_rn(2.f, t), s2);
+              Kn = fmaxf(__fsub_rn(Kr, pj), p.eps);
             }
+            egain[j] = __fsub_rn(base, __fdiv_rn(__fadd_rn(G, dG), __fmul_rn(Kn, Kn)));
           }
         });
       }
