@@ -52,21 +52,63 @@ RESS_DEV int swap_count(int r, int c, float rho, int n_drop) {
   return min(m, min(n_drop, c));
 }
 
-// Applies the chosen swaps to the net drift g (lane holds g[lane], g[lane+32]) and K
-// (Eq. 13 for restores, its mirror for drops): restores in ascending block order, then
-// drops; flags move to KEPT / DROP.  The chosen blocks are first listed in `list` (this
-// warp's shared memory, room for every block), then their rows are fetched eight at a
-// time so that the loads overlap.
-RESS_DEV void apply_swaps(uint8_t *flags, int nb, const float *prow, const float *vph,
-                          float vb0, float vb1, float &g0, float &g1, float &K, int *list) {
+// Adds sg * P_k (vbar - V_k) to the net drift g (lane holds dimensions lane and lane+32)
+// and sk * P_k to ksum for the listed blocks k, in list order.  Rows are fetched eight
+// at a time, and the next eight are requested before the current ones are summed, so
+// that two batches of loads overlap the additions.
+RESS_DEV void gather_drift(const int *list, int n, const float *prow, const float *vph,
+                           float vb0, float vb1, float sg, float sk, float &g0, float &g1,
+                           float &ksum) {
+  const int lane = threadIdx.x & 31;
+  float pk[8], x0[8], x1[8];
+  auto load = [&](int q0, float (&p_)[8], float (&a_)[8], float (&b_)[8]) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int kk = q0 + q < n ? list[q0 + q] : -1;
+      p_[q] = kk >= 0 ? prow[kk] : 0.f;
+      a_[q] = kk >= 0 ? vph[(size_t)kk * kHeadDim + lane] : 0.f;
+      b_[q] = kk >= 0 ? vph[(size_t)kk * kHeadDim + lane + 32] : 0.f;
+    }
+  };
+  if (n > 0) load(0, pk, x0, x1);
+  for (int q0 = 0; q0 < n; q0 += 8) {
+    float pn[8], y0[8], y1[8];
+    if (q0 + 8 < n) load(q0 + 8, pn, y0, y1);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      if (q0 + q < n) {
+        g0 = __fadd_rn(g0, sg * __fmul_rn(pk[q], __fsub_rn(vb0, x0[q])));
+        g1 = __fadd_rn(g1, sg * __fmul_rn(pk[q], __fsub_rn(vb1, x1[q])));
+        ksum = __fadd_rn(ksum, sk * pk[q]);
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      pk[q] = pn[q];
+      x0[q] = y0[q];
+      x1[q] = y1[q];
+    }
+  }
+}
+
+// Applies the chosen swaps to the net drift g and K (Eq. 13 for restores, its mirror
+// for drops): restores in ascending block order, then drops; flags move to KEPT / DROP.
+// The chosen blocks are first listed in `list` (this warp's shared memory, room for
+// every block).  Restores are found by a scan of all nb blocks, drops by a scan of the
+// ascending list of kept candidates (slist, ns entries).
+RESS_DEV void apply_swaps(uint8_t *flags, int nb, const uint16_t *slist, int ns,
+                          const float *prow, const float *vph, float vb0, float vb1, float &g0,
+                          float &g1, float &K, int *list) {
   const int lane = threadIdx.x & 31;
 #pragma unroll 1
   for (int pass = 0; pass < 2; ++pass) {
     const uint8_t target = pass == 0 ? F_TO_KEEP : F_TO_DROP;
+    const int nscan = pass == 0 ? nb : ns;
     int n = 0;
-    for (int c0 = 0; c0 < nb; c0 += 32) {
-      const int j = c0 + lane;
-      const bool sel = j < nb && flags[j] == target;
+    for (int c0 = 0; c0 < nscan; c0 += 32) {
+      const int q = c0 + lane;
+      const int j = q < nscan ? (pass == 0 ? q : (int)slist[q]) : 0;
+      const bool sel = q < nscan && flags[j] == target;
       const unsigned bal = __ballot_sync(0xffffffffu, sel);
       if (sel) {
         list[n + __popc(bal & lanemask_lt())] = j;
@@ -75,32 +117,9 @@ RESS_DEV void apply_swaps(uint8_t *flags, int nb, const float *prow, const float
       n += __popc(bal);
     }
     __syncwarp();
-    for (int q0 = 0; q0 < n; q0 += 8) {
-      float pk[8], x0[8], x1[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const int kk = q0 + q < n ? list[q0 + q] : -1;
-        pk[q] = kk >= 0 ? prow[kk] : 0.f;
-        x0[q] = kk >= 0 ? vph[(size_t)kk * kHeadDim + lane] : 0.f;
-        x1[q] = kk >= 0 ? vph[(size_t)kk * kHeadDim + lane + 32] : 0.f;
-      }
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        if (q0 + q < n) {
-          const float d0 = __fmul_rn(pk[q], __fsub_rn(vb0, x0[q]));
-          const float d1 = __fmul_rn(pk[q], __fsub_rn(vb1, x1[q]));
-          if (pass == 0) {
-            g0 = __fsub_rn(g0, d0);
-            g1 = __fsub_rn(g1, d1);
-            K = __fadd_rn(K, pk[q]);
-          } else {
-            g0 = __fadd_rn(g0, d0);
-            g1 = __fadd_rn(g1, d1);
-            K = __fsub_rn(K, pk[q]);
-          }
-        }
-      }
-    }
+    // restore: g -= P_k e_k, K += P_k; drop: g += P_k e_k, K -= P_k
+    gather_drift(list, n, prow, vph, vb0, vb1, pass == 0 ? -1.f : 1.f, pass == 0 ? 1.f : -1.f,
+                 g0, g1, K);
     __syncwarp();
   }
 }
@@ -131,14 +150,21 @@ RESS_DEV float objective(float G, float K, float eps) {
 }
 
 // Per-warp shared-memory block of the selection kernel: histogram, gather slots, M g,
-// then the row's gain / key array and two flag arrays (current and best drop set).
+// scalars, then the row's gain / key array (nb floats), the flag array (nb bytes) and
+// the best drop set of the restoration rounds as a bitmask (bit j = block j kept).  The
+// CDF method appends nb floats (the kept probabilities in rank order), the restoration
+// rounds an nb-entry list of 16-bit block indices (the kept candidates, ascending).
 // The stride is 16 bytes past a multiple of 128: every warp's block starts 16-byte
-// aligned (float4 reads of M g), and in the cooperative gain pass, where the lanes of
-// one 8-lane phase read M g of eight different rows, those reads fall on distinct banks.
-// The CDF method appends nb floats (the kept probabilities in rank order).
-__host__ __device__ __forceinline__ size_t select_warp_bytes(int nb, bool cdf = false) {
-  const size_t b = 1024 + 128 + 256 + 32 + (size_t)nb * 4 + 2 * (size_t)((nb + 15) & ~15) +
-                   (cdf ? (size_t)nb * 4 : 0);
+// aligned (float4 reads of M g), and the M g reads of eight different rows fall on
+// distinct banks.
+__host__ __device__ __forceinline__ size_t select_flags_bytes(int nb) { return ((size_t)nb + 15) & ~(size_t)15; }
+__host__ __device__ __forceinline__ size_t select_best_bytes(int nb) {
+  return ((((size_t)nb + 31) / 32) * 4 + 15) & ~(size_t)15;
+}
+__host__ __device__ __forceinline__ size_t select_warp_bytes(int nb, bool cdf, bool restore) {
+  const size_t b = 1024 + 128 + 256 + 32 + (size_t)nb * 4 + select_flags_bytes(nb) +
+                   select_best_bytes(nb) + (cdf ? (size_t)nb * 4 : 0) +
+                   (restore ? ((2 * (size_t)nb + 15) & ~(size_t)15) : 0);
   return ((b + 127) & ~(size_t)127) + 16;
 }
 
@@ -162,7 +188,7 @@ __global__ void __launch_bounds__(512) select_kernel(const __grid_constant__ Sel
   float(*sM)[kPad] = reinterpret_cast<float(*)[kPad]>(smem_raw + tile_bytes);
   unsigned char *wbase = smem_raw + tile_bytes + (state ? 64 * kPad * 4 : 0);
   const bool cdf = p.method == RESS_SELECT_CDF;
-  const size_t wbytes = select_warp_bytes(nb, cdf);
+  const size_t wbytes = select_warp_bytes(nb, cdf, restore);
   unsigned char *mine = wbase + wbytes * warp;
   uint32_t *hist = reinterpret_cast<uint32_t *>(mine);
   int *slot = reinterpret_cast<int *>(mine + 1024);
@@ -171,8 +197,19 @@ __global__ void __launch_bounds__(512) select_kernel(const __grid_constant__ Sel
   float *gain = reinterpret_cast<float *>(mine + 1440);
   int *list = reinterpret_cast<int *>(gain);  // block lists reuse the gain array
   uint8_t *flags = mine + 1440 + (size_t)nb * 4;
-  uint8_t *best = flags + ((nb + 15) & ~15);
-  float *sorted = reinterpret_cast<float *>(best + ((nb + 15) & ~15));  // CDF only
+  uint32_t *bestw = reinterpret_cast<uint32_t *>(flags + select_flags_bytes(nb));
+  unsigned char *tail = reinterpret_cast<unsigned char *>(bestw) + select_best_bytes(nb);
+  float *sorted = reinterpret_cast<float *>(tail);      // CDF only
+  uint16_t *slist = reinterpret_cast<uint16_t *>(tail);  // restoration rounds only
+  // the current selection as the best one (bit j of bestw = candidate block j kept)
+  auto save_best = [&]() {
+    for (int c0 = 0; c0 < nb; c0 += 32) {
+      const int j = c0 + lane;
+      const unsigned b = __ballot_sync(0xffffffffu, j < nb && flags[j] == F_KEPT);
+      if (lane == 0) bestw[c0 >> 5] = b;
+    }
+    __syncwarp();
+  };
 
   const long long bh = blockIdx.y;
   const int h = (int)(bh % p.H);
@@ -263,24 +300,7 @@ __global__ void __launch_bounds__(512) select_kernel(const __grid_constant__ Sel
         n += __popc(bal);
       }
       __syncwarp();
-      for (int q0 = 0; q0 < n; q0 += 8) {
-        float pk[8], x0[8], x1[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const int kk = q0 + q < n ? list[q0 + q] : -1;
-          pk[q] = kk >= 0 ? prow[kk] : 0.f;
-          x0[q] = kk >= 0 ? vph[(size_t)kk * kHeadDim + lane] : 0.f;
-          x1[q] = kk >= 0 ? vph[(size_t)kk * kHeadDim + lane + 32] : 0.f;
-        }
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          if (q0 + q < n) {
-            g0 = __fadd_rn(g0, __fmul_rn(pk[q], __fsub_rn(vb0, x0[q])));
-            g1 = __fadd_rn(g1, __fmul_rn(pk[q], __fsub_rn(vb1, x1[q])));
-            Psum = __fadd_rn(Psum, pk[q]);
-          }
-        }
-      }
+      gather_drift(list, n, prow, vph, vb0, vb1, 1.f, 1.f, g0, g1, Psum);
       __syncwarp();
       if (kept_form) {
         g0 = -g0;
@@ -292,10 +312,7 @@ __global__ void __launch_bounds__(512) select_kernel(const __grid_constant__ Sel
     float G = gather ? gram_apply(sM, g0, g1, h0, h1) : 0.f;
     float J = objective(G, K, p.eps);
     float bestJ = J;
-    if (work) {
-      for (int j = lane; j < nb; j += 32) best[j] = flags[j];
-      __syncwarp();
-    }
+    if (work) save_best();
 #pragma unroll 1
     for (int r = 0; r < p.rounds; ++r) {
       const int m = swap_count(r, c, p.rho, n_drop);
@@ -428,20 +445,34 @@ __global__ void __launch_bounds__(512) select_kernel(const __grid_constant__ Sel
         auto gkey = [&](int j) { return float_key(maximise ? -gain[j] : gain[j]); };
         warp_select<uint32_t>(nb, m, gkey, [&](int j) { return flags[j] == F_DROP; },
                              [&](int j) { flags[j] = F_TO_KEEP; }, hist, slot);
-        warp_select<uint32_t>(nb, m, gkey, [&](int j) { return flags[j] == F_KEPT; },
-                             [&](int j) { flags[j] = F_TO_DROP; }, hist, slot);
-        apply_swaps(flags, nb, prow, vph, vb0, vb1, g0, g1, K, list);
+        // the kept candidates S as an ascending list: the drop-side select and the drop
+        // pass of apply_swaps walk |S| entries instead of nb
+        int ns = 0;
+        for (int c0 = 0; c0 < nb; c0 += 32) {
+          const int j = c0 + lane;
+          const bool sel = j < nb && flags[j] == F_KEPT;
+          const unsigned bal = __ballot_sync(0xffffffffu, sel);
+          if (sel) slist[ns + __popc(bal & lanemask_lt())] = (uint16_t)j;
+          ns += __popc(bal);
+        }
+        __syncwarp();
+        warp_select<uint32_t>(ns, m, [&](int q) { return gkey(slist[q]); },
+                             [&](int q) { return flags[slist[q]] == F_KEPT; },
+                             [&](int q) { flags[slist[q]] = F_TO_DROP; }, hist, slot);
+        apply_swaps(flags, nb, slist, ns, prow, vph, vb0, vb1, g0, g1, K, list);
         G = gram_apply(sM, g0, g1, h0, h1);
         J = objective(G, K, p.eps);
         if (maximise ? J > bestJ : J < bestJ) {  // track-best (track-worst when maximising)
           bestJ = J;
-          for (int j = lane; j < nb; j += 32) best[j] = flags[j];
-          __syncwarp();
+          save_best();
         }
       }
     }
     if (work) {
-      for (int j = lane; j < nb; j += 32) flags[j] = best[j];
+      for (int j = lane; j < nb; j += 32) {
+        const uint8_t f = flags[j];
+        if (f == F_KEPT || f == F_DROP) flags[j] = (bestw[j >> 5] >> (j & 31)) & 1u ? F_KEPT : F_DROP;
+      }
       __syncwarp();
     }
     // realized drift of the returned selection ([ReSS] §6.1): the tracked J after the
@@ -579,7 +610,7 @@ __global__ void __launch_bounds__(1024) schedule_kernel_par(const int32_t *__res
 
 static size_t select_smem(int nb, int T, bool restore, bool state, bool cdf) {
   return (restore ? (size_t)kSelStages * kTileFloats * 4 : 0) + (state ? 64 * kPad * 4 : 0) +
-         select_warp_bytes(nb, cdf) * T;
+         select_warp_bytes(nb, cdf, restore) * T;
 }
 
 cudaError_t launch_select(const Dims &d, const SelectLaunch &a, cudaStream_t st) {

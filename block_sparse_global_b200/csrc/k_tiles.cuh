@@ -41,12 +41,15 @@ RESS_DEV void tile_load(float *dst, const float *src, int t, int nb) {
 }
 
 // Walks all tiles of `src` through `Stages` buffers (Stages * kTileFloats floats at
-// `buf`), keeping Stages - 1 tile loads in flight, and calls body(t, tile) once per tile
-// with the whole CTA synchronised around each call.  body must not write the buffers.
-// Exactly one cp.async group is committed per tile slot (empty past the last tile), so
-// waiting for all but the newest Stages - 1 groups always covers tile t.
+// `buf`), keeping up to Stages - 1 tile loads in flight, and calls body(t, tile) once
+// per tile with the whole CTA synchronised before each call.  One barrier per tile: the
+// refill of the buffer that tile t - 1 used is issued only after that barrier, when
+// every thread has finished body(t - 1).  Exactly one cp.async group is committed per
+// tile slot (empty past the last tile), so waiting for all but the newest Stages - 2
+// groups always covers tile t.  body must not write the buffers.
 template <int Stages, typename Body>
 RESS_DEV void tile_stream_n(float *buf, const float *src, int nb, Body body) {
+  static_assert(Stages >= 2, "at least two buffers");
   const int ntiles = (nb + kTileKeys - 1) / kTileKeys;
   __syncthreads();  // buffers free (previous users done)
 #pragma unroll
@@ -55,14 +58,14 @@ RESS_DEV void tile_stream_n(float *buf, const float *src, int nb, Body body) {
     else cp_async_commit();
   }
   for (int t = 0; t < ntiles; ++t) {
+    cp_async_wait<Stages - 2>();
+    __syncthreads();  // tile t visible to all; everyone is done with tile t - 1
     const int tn = t + Stages - 1;
     if (tn < ntiles) tile_load(buf + (tn % Stages) * kTileFloats, src, tn, nb);
     else cp_async_commit();
-    cp_async_wait<Stages - 1>();
-    __syncthreads();  // tile t visible to all
     body(t, buf + (t % Stages) * kTileFloats);
-    __syncthreads();  // everyone done with tile t before its buffer is reloaded
   }
+  __syncthreads();  // the buffers are free again when the walk returns
 }
 
 // Two-buffer form used by the block-map and drift kernels.
