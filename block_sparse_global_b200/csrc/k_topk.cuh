@@ -55,9 +55,8 @@ RESS_DEV void warp_top_k(int n, int k, KeyFn key, ValidFn valid, MarkFn mark, ui
         in = hi_shift >= BITS || (kk >> hi_shift) == (prefix >> hi_shift);
         bin = (uint32_t)(kk >> shift) & 255u;
       }
-      // lanes with the same bin add once, through their lowest lane
-      const unsigned peers = __match_any_sync(0xffffffffu, in ? bin : 256u);
-      if (in && (peers & lanemask_lt()) == 0) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+      // shared-memory atomics resolve lanes that hit the same bin in hardware
+      if (in) atomicAdd(&hist[bin], 1u);
     }
     __syncwarp();
     // lane l holds bins 255-8l .. 248-8l (highest digits first)
