@@ -201,26 +201,63 @@ __global__ void __launch_bounds__(kThreads) block_scores_kernel(
     const int r = idx / kHeadDim;
     sq[idx] = (i0 + r < nq) ? qh[(size_t)(i0 + r) * kHeadDim + idx % kHeadDim] : 0.f;
   }
-  // logits: lane takes key blocks lane and lane + 32 of each tile
-  tile_stream(tiles, kp + (size_t)bh * nk * kHeadDim, nk, [&](int tt, const float *tile) {
-    const float4 *k0 = reinterpret_cast<const float4 *>(tile + lane * kTilePad);
-    const float4 *k1 = reinterpret_cast<const float4 *>(tile + (lane + 32) * kTilePad);
+  // logits: thread t takes a 4-row x (TQ/2)-block micro-tile (row group rg, block group
+  // kg) of each 64-block tile over 8 of the 64 dimensions (slice ds: 4ds..4ds+3 and
+  // 32+4ds..32+4ds+3), with its rows' pooled-query slices in registers; the 8 slices of
+  // a micro-tile sit on 8 consecutive lanes and a transposing butterfly (xor 4, 2, 1)
+  // sums them, leaving lane ds the TQ/4 logits of row ds/2, blocks (TQ/4)(ds%2) + i.
+  {
+    constexpr int KPM = TQ / 2, NV = TQ / 4, NRG = TQ / 4;
+    const int ds = t & 7, mt = t >> 3;  // 32 micro-tiles
+    const int rg = mt % NRG, kg = mt / NRG;
+    __syncthreads();  // pooled queries staged
+    float4 qv[4][2];
 #pragma unroll
-    for (int q = 0; q < R; ++q) {
-      const int r = warp * R + q;
-      const float4 *qq = reinterpret_cast<const float4 *>(sq + r * kHeadDim);
-      float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-      for (int d = 0; d < 16; ++d) {
-        const float4 x = qq[d], y0 = k0[d], y1 = k1[d];
-        a0 = fmaf(x.x, y0.x, a0); a0 = fmaf(x.y, y0.y, a0); a0 = fmaf(x.z, y0.z, a0); a0 = fmaf(x.w, y0.w, a0);
-        a1 = fmaf(x.x, y1.x, a1); a1 = fmaf(x.y, y1.y, a1); a1 = fmaf(x.z, y1.z, a1); a1 = fmaf(x.w, y1.w, a1);
-      }
-      const int j = tt * kTileKeys + lane;
-      if (j < nk) sl[r * nk + j] = a0 * scale;
-      if (j + 32 < nk) sl[r * nk + j + 32] = a1 * scale;
+    for (int r = 0; r < 4; ++r) {
+      const float4 *qr = reinterpret_cast<const float4 *>(sq + (rg * 4 + r) * kHeadDim);
+      qv[r][0] = qr[ds];
+      qv[r][1] = qr[8 + ds];
     }
-  });
+    const bool b2 = ds & 4, b1 = ds & 2, b0 = ds & 1;
+    float *lrow = sl + (rg * 4 + (ds >> 1)) * nk;
+    const int jq = kg * KPM + NV * (ds & 1);
+    tile_stream(tiles, kp + (size_t)bh * nk * kHeadDim, nk, [&](int tt, const float *tile) {
+      float acc[4 * KPM];
+#pragma unroll
+      for (int kk = 0; kk < KPM; ++kk) {
+        const float4 *vk = reinterpret_cast<const float4 *>(tile + (kg * KPM + kk) * kTilePad);
+        const float4 a = vk[ds], b = vk[8 + ds];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const float4 x = qv[r][0], y = qv[r][1];
+          float d = a.x * x.x;
+          d = fmaf(a.y, x.y, d); d = fmaf(a.z, x.z, d); d = fmaf(a.w, x.w, d);
+          d = fmaf(b.x, y.x, d); d = fmaf(b.y, y.y, d); d = fmaf(b.z, y.z, d); d = fmaf(b.w, y.w, d);
+          acc[r * KPM + kk] = d;
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 2 * KPM; ++i) {
+        const float send = b2 ? acc[i] : acc[2 * KPM + i], keep = b2 ? acc[2 * KPM + i] : acc[i];
+        acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+      }
+#pragma unroll
+      for (int i = 0; i < KPM; ++i) {
+        const float send = b1 ? acc[i] : acc[KPM + i], keep = b1 ? acc[KPM + i] : acc[i];
+        acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+      }
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        const float send = b0 ? acc[i] : acc[NV + i], keep = b0 ? acc[NV + i] : acc[i];
+        acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+      }
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        const int j = tt * kTileKeys + jq + i;
+        if (j < nk) lrow[j] = acc[i] * scale;
+      }
+    });
+  }
   // softmax over every key block, per row
 #pragma unroll
   for (int q = 0; q < R; ++q) {
@@ -307,30 +344,40 @@ __global__ void __launch_bounds__(kThreads) block_scores_kernel(
     }
     if (vbar == nullptr) return;
   }
-  // vbar_i = sum_j P_ij V_j: lane takes value dimensions lane and lane + 32
-  float a0[R], a1[R];
+  // vbar_i = sum_j P_ij V_j.  Warp w takes blocks w, w + 8, ... of each tile for all TQ
+  // rows (lane: value dimensions lane and lane + 32), so that one read of a pooled-value
+  // row serves every row of the CTA; the eight warps' partial sums then meet in shared
+  // memory (the tile buffers, free once the walk is over) and are added in warp order.
+  float a0[TQ], a1[TQ];
 #pragma unroll
-  for (int q = 0; q < R; ++q) a0[q] = a1[q] = 0.f;
+  for (int q = 0; q < TQ; ++q) a0[q] = a1[q] = 0.f;
   tile_stream(tiles, vp + (size_t)bh * nk * kHeadDim, nk, [&](int tt, const float *tile) {
     const int jn = min(kTileKeys, nk - tt * kTileKeys);
+    for (int kk = warp; kk < jn; kk += kWarps) {
+      const float x0 = tile[kk * kTilePad + lane], x1 = tile[kk * kTilePad + lane + 32];
+      const float *pc = sl + tt * kTileKeys + kk;
 #pragma unroll
-    for (int q = 0; q < R; ++q) {
-      const float *row = sl + (warp * R + q) * nk + tt * kTileKeys;
-      for (int kk = 0; kk < jn; ++kk) {
-        const float pj = row[kk];
-        a0[q] = fmaf(pj, tile[kk * kTilePad + lane], a0[q]);
-        a1[q] = fmaf(pj, tile[kk * kTilePad + lane + 32], a1[q]);
+      for (int q = 0; q < TQ; ++q) {
+        const float pj = pc[q * nk];
+        a0[q] = fmaf(pj, x0, a0[q]);
+        a1[q] = fmaf(pj, x1, a1[q]);
       }
     }
   });
+  float *part = tiles;  // [kWarps][TQ][64], within the two tile buffers
+  static_assert(kWarps * TQ * kHeadDim <= 2 * kTileFloats, "partials fit in the tile buffers");
 #pragma unroll
-  for (int q = 0; q < R; ++q) {
-    const int i = i0 + warp * R + q;
-    if (i < nq) {
-      float *o = vbar + ((size_t)bh * nq + i) * kHeadDim;
-      o[lane] = a0[q];
-      o[lane + 32] = a1[q];
-    }
+  for (int q = 0; q < TQ; ++q) {
+    part[(warp * TQ + q) * kHeadDim + lane] = a0[q];
+    part[(warp * TQ + q) * kHeadDim + lane + 32] = a1[q];
+  }
+  __syncthreads();
+  for (int idx = t; idx < TQ * kHeadDim; idx += kThreads) {
+    const int q = idx / kHeadDim, i = i0 + q;
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) v += part[w * TQ * kHeadDim + idx];
+    if (i < nq) vbar[((size_t)bh * nq + i) * kHeadDim + idx % kHeadDim] = v;
   }
 }
 
