@@ -422,50 +422,79 @@ __global__ void __launch_bounds__(kThreads) drift_prep_kernel(
   }
 }
 
-// Pass 2: s_ij = P_ij sqrt(max(a_i - 2 w_i . V_j + c_j, 0)).  One CTA per (b*h, 16 rows),
-// two rows per warp; the head's pooled values stream through shared memory in tiles of
-// 64 blocks, lane = key block (lane and lane + 32).
+// Pass 2: s_ij = P_ij sqrt(max(a_i - 2 w_i . V_j + c_j, 0)).  One CTA per (b*h, 16 rows);
+// the head's pooled values stream through shared memory in tiles of 64 blocks.  Thread
+// t takes a 4-row x 8-block micro-tile of each tile over 8 of the 64 dimensions (slice
+// ds: 4ds..4ds+3 and 32+4ds..32+4ds+3), with its rows' w slices in registers; the 8
+// slices of a micro-tile sit on 8 consecutive lanes and a transposing butterfly (xor 4,
+// 2, 1) sums them, leaving lane ds the inner products of row ds/2 with blocks
+// 4(ds%2) .. 4(ds%2)+3, whose scores it writes.
 constexpr int kDriftRows = 16;
 __global__ void __launch_bounds__(kThreads) drift_kernel(
     const float *__restrict__ P, const float *__restrict__ vp, const float *__restrict__ w,
     const float *__restrict__ a, const float *__restrict__ c, float *__restrict__ s, int nq, int nk) {
-  constexpr int R = kDriftRows / kWarps;
+  constexpr int KPM = 8, NV = 4, NRG = kDriftRows / 4;
+  static_assert(NRG * (kTileKeys / KPM) * 8 == kThreads, "one micro-tile slice per thread");
   __shared__ __align__(16) float tiles[2 * kTileFloats];
   __shared__ __align__(16) float sw[kDriftRows][kHeadDim];
-  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int t = threadIdx.x;
   const long long bh = blockIdx.y;
   const int i0 = blockIdx.x * kDriftRows;
   for (int idx = t; idx < kDriftRows * kHeadDim; idx += kThreads) {
     const int r = idx / kHeadDim;
     sw[r][idx % kHeadDim] = (i0 + r < nq) ? w[((size_t)bh * nq + i0 + r) * kHeadDim + idx % kHeadDim] : 0.f;
   }
-  float ai[R];
+  const int ds = t & 7, mt = t >> 3;
+  const int rg = mt % NRG, kg = mt / NRG;
+  __syncthreads();  // w rows staged
+  float4 wv[4][2];
 #pragma unroll
-  for (int q = 0; q < R; ++q) {
-    const int i = i0 + warp * R + q;
-    ai[q] = i < nq ? a[(size_t)bh * nq + i] : 0.f;
+  for (int r = 0; r < 4; ++r) {
+    const float4 *wr = reinterpret_cast<const float4 *>(&sw[rg * 4 + r][0]);
+    wv[r][0] = wr[ds];
+    wv[r][1] = wr[8 + ds];
   }
+  const int ie = i0 + rg * 4 + (ds >> 1);  // the row whose scores this lane writes
+  const float ae = ie < nq ? a[(size_t)bh * nq + ie] : 0.f;
+  const size_t orow = ((size_t)bh * nq + (ie < nq ? ie : 0)) * nk;
+  const int jq = kg * KPM + NV * (ds & 1);
   const float *ch = c + (size_t)bh * nk;
+  const bool b2 = ds & 4, b1 = ds & 2, b0 = ds & 1;
   tile_stream(tiles, vp + (size_t)bh * nk * kHeadDim, nk, [&](int tt, const float *tile) {
-    const float4 *v0 = reinterpret_cast<const float4 *>(tile + lane * kTilePad);
-    const float4 *v1 = reinterpret_cast<const float4 *>(tile + (lane + 32) * kTilePad);
-    const int j0 = tt * kTileKeys + lane, j1 = j0 + 32;
-    const float c0 = j0 < nk ? ch[j0] : 0.f, c1 = j1 < nk ? ch[j1] : 0.f;
+    float acc[4 * KPM];
 #pragma unroll
-    for (int q = 0; q < R; ++q) {
-      const int r = warp * R + q, i = i0 + r;
-      const float4 *ww = reinterpret_cast<const float4 *>(&sw[r][0]);
-      float d0 = 0.f, d1 = 0.f;
-#pragma unroll 4
-      for (int d = 0; d < 16; ++d) {
-        const float4 x = ww[d], y0 = v0[d], y1 = v1[d];
-        d0 = fmaf(x.x, y0.x, d0); d0 = fmaf(x.y, y0.y, d0); d0 = fmaf(x.z, y0.z, d0); d0 = fmaf(x.w, y0.w, d0);
-        d1 = fmaf(x.x, y1.x, d1); d1 = fmaf(x.y, y1.y, d1); d1 = fmaf(x.z, y1.z, d1); d1 = fmaf(x.w, y1.w, d1);
+    for (int kk = 0; kk < KPM; ++kk) {
+      const float4 *vk = reinterpret_cast<const float4 *>(tile + (kg * KPM + kk) * kTilePad);
+      const float4 x = vk[ds], y = vk[8 + ds];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const float4 u = wv[r][0], v = wv[r][1];
+        float d = u.x * x.x;
+        d = fmaf(u.y, x.y, d); d = fmaf(u.z, x.z, d); d = fmaf(u.w, x.w, d);
+        d = fmaf(v.x, y.x, d); d = fmaf(v.y, y.y, d); d = fmaf(v.z, y.z, d); d = fmaf(v.w, y.w, d);
+        acc[r * KPM + kk] = d;
       }
-      if (i < nq) {
-        const size_t o = ((size_t)bh * nq + i) * nk;
-        if (j0 < nk) s[o + j0] = P[o + j0] * sqrtf(fmaxf((ai[q] - 2.f * d0) + c0, 0.f));
-        if (j1 < nk) s[o + j1] = P[o + j1] * sqrtf(fmaxf((ai[q] - 2.f * d1) + c1, 0.f));
+    }
+#pragma unroll
+    for (int i = 0; i < 2 * KPM; ++i) {
+      const float send = b2 ? acc[i] : acc[2 * KPM + i], keep = b2 ? acc[2 * KPM + i] : acc[i];
+      acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+    }
+#pragma unroll
+    for (int i = 0; i < KPM; ++i) {
+      const float send = b1 ? acc[i] : acc[KPM + i], keep = b1 ? acc[KPM + i] : acc[i];
+      acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+    }
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const float send = b0 ? acc[i] : acc[NV + i], keep = b0 ? acc[NV + i] : acc[i];
+      acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+    }
+    if (ie < nq) {
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        const int j = tt * kTileKeys + jq + i;
+        if (j < nk) s[orow + j] = P[orow + j] * sqrtf(fmaxf((ae - 2.f * acc[i]) + ch[j], 0.f));
       }
     }
   });
