@@ -56,6 +56,8 @@ def parse():
                     help="drift objective: the method, or a drift-maximising control (drift only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-groups", type=int, default=4,
+                    help="head groups of the host-buffer call (copy in / kernels / copy out overlap)")
     ap.add_argument("--quick", action="store_true", help="timed loop only (profiling runs)")
     ap.add_argument("--sweep", action="store_true",
                     help="64-view sweep: sparsity {0,25,50,75,90}%% x {mass, drift, random} over "
@@ -337,7 +339,7 @@ def run_ours(args):
             outh = torch.empty(layer.out.shape, dtype=layer.out.dtype).pin_memory()
             qd, kd, vd = (torch.empty_like(x) for x in (q, k, v))
             # head groups: copies in, kernels and copies out overlap on three streams
-            groups = 1 if wl.method == R.SELECT_RANDOM else 4
+            groups = 1 if wl.method == R.SELECT_RANDOM else max(1, min(args.e2e_groups, H))
             layer.make_groups(wl.w_o, groups)
             e2e_ms = []
             for s in range(max(3, args.steps // 2) + 2):
