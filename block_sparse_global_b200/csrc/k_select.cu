@@ -646,6 +646,16 @@ cudaError_t launch_select(const Dims &d, const SelectLaunch &a, cudaStream_t st)
   int T = restore ? 16 : 4;
   const bool cdf = a.method == RESS_SELECT_CDF;
   while (T > 4 && select_smem(d.nk, T, restore, state, cdf) > 220 * 1024) T >>= 1;
+  if (restore && T == 16) {
+    // 8 rows per CTA when that fits two CTAs per SM (small nb): the same 16 warps per SM
+    // in finer CTAs, whose barriers and last wave cost less (32 views: -6 %)
+    int dev = 0, per_sm = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) ==
+            cudaSuccess &&
+        2 * (select_smem(d.nk, 8, restore, state, cdf) + 1024) <= (size_t)per_sm)
+      T = 8;
+  }
   p.rows_per_cta = T;
   const size_t smem = select_smem(d.nk, T, restore, state, cdf);
   cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
