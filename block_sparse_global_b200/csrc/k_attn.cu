@@ -66,10 +66,12 @@ struct Bars {
   uint64_t p_full;
   uint64_t o_done;
   uint64_t drain;
+  uint64_t never;  // completed by nobody: the diagnostic stall of stall_cycles waits here
   uint32_t tmem_base;
   int abort;
   int row_state;  // 0 = run, 1 = empty row (kv_cnt == 0), 2 = invalid row
 };
+static_assert(sizeof(Bars) <= 256, "barriers fit their shared-memory slot");
 
 // Shared-memory matrix descriptor, 128-byte swizzle, 8-row groups 1024 bytes apart.
 RESS_DEV uint64_t smem_desc(uint32_t saddr) {
@@ -145,6 +147,7 @@ struct AttnParams {
   int N, nq, nk;  // tokens; query and key blocks per (batch, head)
   long long items;
   float scale_log2;
+  long long stall_cycles;  // > 0 only for ress_debug_attn_forced_timeout
 };
 
 // KB = tokens per key block (128 or 64); a score tile always spans 128 keys.
@@ -181,6 +184,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     mbar_init(&bar->p_full, 4);
     mbar_init(&bar->o_done, 1);
     mbar_init(&bar->drain, 1);
+    mbar_init(&bar->never, 1);
     bar->abort = 0;
     fence_mbar_init();
   }
@@ -316,6 +320,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int last_valid = p.N - (p.nk - 1) * KB;  // tokens in the last key block
       float m_run = -INFINITY, l_run = 0.f;
       bool ok = true;
+      // diagnostics only: wait, with the given limit, on a barrier that nothing
+      // completes, so that the CTA takes the bounded-wait timeout path below (error word,
+      // producer and MMA warps released through `abort`, copies and MMAs drained)
+      if (p.stall_cycles > 0) ok = mbar_wait_for(&bar->never, 0, abort, p.stall_cycles);
       // kept block(s) of the next tile, read ahead of the barrier wait
       int kb_next = kvrow[0];
       int kb2_next = KB == 64 ? (cnt > 1 ? kvrow[1] : -1) : -1;
@@ -508,6 +516,7 @@ cudaError_t launch_attn(const Dims &d, const AttnLaunch &a, cudaStream_t st) {
   p.nk = d.nk;
   p.items = d.BH() * d.nq;
   p.scale_log2 = a.scale * 1.4426950408889634f;
+  p.stall_cycles = a.stall_cycles;
   auto kern = d.kb == 64 ? attn_kernel<64> : attn_kernel<128>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);

@@ -284,6 +284,38 @@ ress_status ress_block_sparse_attn(const ress_shape *shape, const void *q, const
   return from_cuda(e);
 }
 
+ress_status ress_debug_attn_forced_timeout(const ress_shape *shape, const void *q, const void *k,
+                                           const void *v, const int32_t *kv_idx,
+                                           const int32_t *kv_cnt, float scale, void *out,
+                                           int32_t *dev_err, int64_t limit_cycles,
+                                           ress_stream_t stream) {
+  if (limit_cycles <= 0 || limit_cycles > (int64_t)1 << 32) return RESS_ERR_INVALID_ARG;
+  if (dev_err == nullptr || (reinterpret_cast<uintptr_t>(dev_err) & 3u)) return RESS_ERR_INVALID_ARG;
+  Dims d;
+  bool empty;
+  ress_status st = check_shape(shape, &d, &empty);
+  if (st != RESS_OK) return st;
+  if (empty) return RESS_OK;
+  if (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(v) || !ptr_ok(kv_idx) || !ptr_ok(kv_cnt) || !ptr_ok(out))
+    return RESS_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || scale != scale) return RESS_ERR_INVALID_ARG;
+  ress::AttnLaunch a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.kv_idx = kv_idx;
+  a.kv_cnt = kv_cnt;
+  a.order = nullptr;
+  a.scale = scale;
+  a.out = out;
+  a.lse = nullptr;
+  a.dev_err = dev_err;
+  a.stall_cycles = (long long)limit_cycles;
+  cudaError_t e = ress::launch_attn(d, a, (cudaStream_t)stream);
+  if (e == cudaErrorNotSupported) return RESS_ERR_CUDA;
+  return from_cuda(e);
+}
+
 }  // extern "C"
 
 // ---------------------------------------------------------------------------------------

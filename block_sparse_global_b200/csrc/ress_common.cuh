@@ -87,16 +87,20 @@ RESS_DEV bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 // Waits for the phase of `bar` with the given parity to complete.  Returns false if the
 // wait gave up (time limit, or *abort became non-zero meanwhile); both are checked every
 // 64 polls so that a waiting warp issues little besides the poll itself.
-RESS_DEV bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+RESS_DEV bool mbar_wait_for(uint64_t *bar, uint32_t parity, volatile int *abort,
+                            long long limit_cycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 63u) == 0) {
       if (abort != nullptr && *abort) return false;
-      if (clock64() - t0 > RESS_WAIT_LIMIT_CYCLES) return false;
+      if (clock64() - t0 > limit_cycles) return false;
     }
   }
+}
+RESS_DEV bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+  return mbar_wait_for(bar, parity, abort, RESS_WAIT_LIMIT_CYCLES);
 }
 
 // ------------------------------------------------------------------------------- TMA

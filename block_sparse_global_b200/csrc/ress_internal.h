@@ -71,6 +71,7 @@ struct AttnLaunch {
   void *out;
   float *lse;
   int32_t *dev_err;
+  long long stall_cycles = 0;  // > 0: the diagnostic forced timeout
 };
 // Returns cudaErrorNotSupported if the driver cannot encode tensor maps.
 cudaError_t launch_attn(const Dims &d, const AttnLaunch &a, cudaStream_t st);

@@ -68,6 +68,9 @@ _SIGS = {
     "ress_attn_schedule": (_I32, [ctypes.POINTER(ress_shape), _VP, _VP, _VP]),
     "ress_block_sparse_attn": (_I32, [ctypes.POINTER(ress_shape), _VP, _VP, _VP, _VP, _VP, _VP,
                                       ctypes.c_float, _VP, _VP, _VP, _VP]),
+    "ress_debug_attn_forced_timeout": (_I32, [ctypes.POINTER(ress_shape), _VP, _VP, _VP, _VP,
+                                              _VP, ctypes.c_float, _VP, _VP, ctypes.c_int64,
+                                              _VP]),
 }
 
 
@@ -233,3 +236,15 @@ def ress_block_sparse_attn(shape, q, k, v, kv_idx, kv_cnt, work_order, scale: fl
                                        _ptr(kv_idx), _ptr(kv_cnt), _ptr(work_order), float(scale),
                                        _ptr(out), _ptr(lse), _ptr(dev_err), _stream(stream))
     _check("ress_block_sparse_attn", st)
+
+
+def ress_debug_attn_forced_timeout(shape, q, k, v, kv_idx, kv_cnt, scale: float, out, dev_err,
+                                   limit_cycles: int, stream=None):
+    """Diagnostics of the device error path (see include/ress.h): the attention kernel with
+    every CTA's softmax stalled on a barrier that nothing completes, so that each takes its
+    bounded-wait timeout path and writes RESS_ERR_DEVICE_TIMEOUT to dev_err."""
+    st = load().ress_debug_attn_forced_timeout(ctypes.byref(_shape(shape)), _ptr(q), _ptr(k),
+                                               _ptr(v), _ptr(kv_idx), _ptr(kv_cnt), float(scale),
+                                               _ptr(out), _ptr(dev_err), int(limit_cycles),
+                                               _stream(stream))
+    _check("ress_debug_attn_forced_timeout", st)

@@ -336,6 +336,26 @@ ress_status ress_block_sparse_attn(const ress_shape *shape, const void *q, const
                                    float scale, void *out, float *lse, int32_t *dev_err,
                                    ress_stream_t stream);
 
+/*
+ * ress_debug_attn_forced_timeout -- diagnostics for the device error path; the pages have
+ * no counterpart.  Launches the same attention kernel as ress_block_sparse_attn (same
+ * arguments, no work_order, no lse), except that every CTA's softmax warps first wait on
+ * an internal barrier that nothing ever completes, giving up after `limit_cycles` SM
+ * clock cycles (1 .. 2^32; about 0.5 ms per million cycles at 2 GHz).  Each CTA then
+ * takes the path a genuinely stuck wait would take: RESS_ERR_DEVICE_TIMEOUT is written to
+ * *dev_err (required here), the TMA and MMA warps are released, every copy and MMA
+ * already issued is drained, tensor memory is freed, and the CTA exits without trapping;
+ * `out` is left unwritten.  The CUDA context stays usable: a following normal call
+ * computes normally.  Host validation as for ress_block_sparse_attn, plus
+ * RESS_ERR_INVALID_ARG for a NULL or misaligned dev_err or a limit out of range.
+ * For tests of the error path; never needed to compute attention.
+ */
+ress_status ress_debug_attn_forced_timeout(const ress_shape *shape, const void *q,
+                                           const void *k, const void *v,
+                                           const int32_t *kv_idx, const int32_t *kv_cnt,
+                                           float scale, void *out, int32_t *dev_err,
+                                           int64_t limit_cycles, ress_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -172,3 +172,19 @@ def test_python_binding_raises(lib):
     with pytest.raises(R.RessError) as e:
         R.ress_attn_schedule(R.make_shape(1, 4, 1024, head_dim=32), None, None)
     assert e.value.status == UNSUPPORTED
+
+
+def test_forced_timeout_diagnostic_validation(lib):
+    """The diagnostic entry point validates like the attention call, and needs a dev_err
+    word and a positive, bounded wait limit (checked on the host, nothing launched)."""
+    shape = ctypes.byref(R.make_shape(1, 2, 1024))
+    args = [FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.c_float(0.125), FAKE]
+    i64 = ctypes.c_int64
+    assert lib.ress_debug_attn_forced_timeout(shape, *args, None, i64(1000), None) == INVALID
+    assert lib.ress_debug_attn_forced_timeout(shape, *args, FAKE + 2, i64(1000), None) == INVALID
+    assert lib.ress_debug_attn_forced_timeout(shape, *args, FAKE, i64(0), None) == INVALID
+    assert lib.ress_debug_attn_forced_timeout(shape, *args, FAKE, i64(-5), None) == INVALID
+    assert lib.ress_debug_attn_forced_timeout(shape, *args, FAKE, i64((1 << 32) + 1), None) == INVALID
+    bad = [FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.c_float(0.0), FAKE]
+    assert lib.ress_debug_attn_forced_timeout(shape, *bad, FAKE, i64(1000), None) == INVALID
+    assert lib.ress_debug_attn_forced_timeout(None, *args, FAKE, i64(1000), None) == INVALID
