@@ -63,6 +63,9 @@ def parse():
                     help="64-view sweep: sparsity {0,25,50,75,90}%% x {mass, drift, random} over "
                          "--layers independent layers, one JSON line per point (not the bench line)")
     ap.add_argument("--layers", type=int, default=24, help="layers of the --sweep")
+    ap.add_argument("--sweep-out", default=None,
+                    help="JSONL file the --sweep appends each finished point to; points already "
+                         "in it are skipped (resume)")
     return ap.parse_args()
 
 
@@ -488,14 +491,34 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def sweep_todo(path, methods, sparsities, key_block: int, layers: int):
+    """The (method name, method, sparsity) points of the sweep still to run: every point
+    minus those already recorded in the JSONL file `path` (same key block and layer count).
+    Lines that do not parse (a run cut off mid-write) are ignored."""
+    done = set()
+    if path and os.path.exists(path):
+        with open(path) as f:
+            for line in f:
+                try:
+                    d = json.loads(line)
+                    c = d["config"]
+                    done.add((c["method"], float(c["sparsity"]), int(c["key_block"]), int(d["layers"])))
+                except (ValueError, KeyError, TypeError):
+                    continue
+    return [(mn, m, sp) for mn, m in methods for sp in sparsities
+            if (mn, float(sp), int(key_block), int(layers)) not in done]
+
+
 def run_sweep(args):
-    """The 64-view sweep: for each of `layers` layers (independent seeded Q, K, V, W_O),
-    every (method, sparsity) point runs the whole path (pool, block map, drift for the
-    drift method, selection, schedule, attention): one warm-up step, then two timed steps,
-    each after an L2 flush.  One JSON line per point: mean layer latency over the layers
-    and kept-tile TFLOP/s (kept-tile FLOPs of all timed steps / their summed device time).
+    """The 64-view sweep: `layers` layers (independent seeded Q, K, V, W_O, all resident in
+    HBM, about 0.55 GB each) and, for each (method, sparsity) point in turn, the whole path
+    (pool, block map, drift for the drift method, selection, schedule, attention) on every
+    layer: one warm-up step, then two timed steps, each after an L2 flush.  One JSON line
+    per point, printed as soon as the point is done: mean layer latency over the layers and
+    kept-tile TFLOP/s (kept-tile FLOPs of all timed steps / their summed device time).
     Sparsity 0 keeps every key block: the same-shape dense layer through the same kernels.
-    Single GPU only (rank 0)."""
+    With --sweep-out FILE each line is also appended to FILE, and points already in FILE
+    are skipped, so an interrupted sweep resumes at the next point.  Single GPU (rank 0)."""
     import torch
 
     from block_sparse_global_b200 import build as B
@@ -511,82 +534,79 @@ def run_sweep(args):
     torch.cuda.set_device(dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, device=dev, dtype=torch.float32)
     methods = [("mass", R.SELECT_MASS), ("drift", R.SELECT_DRIFT), ("random", R.SELECT_RANDOM)]
-    acc = {}
-    layer = None
+    todo = sweep_todo(args.sweep_out, methods, W.SWEEP_SPARSITIES, args.key_block, args.layers)
+    if not todo:
+        return
+    wls = [W.make_workload(5, layer=li, device="cuda", key_block=args.key_block)
+           for li in range(args.layers)]
+    Bsz, H, N, _ = wls[0].q.shape
+    layer = SparseGlobalAttention(Bsz, H, N, device=dev, key_block=args.key_block)
+    n_cand = layer.nk - int(wls[0].keep_k.sum().item())
     sdpa_ms = None
-    clocks = ClockSampler(0)
-    clocks.start()
-    for li in range(args.layers):
-        wl = W.make_workload(5, layer=li, device="cuda", key_block=args.key_block)
-        Bsz, H, N, _ = wl.q.shape
-        if layer is None:
-            layer = SparseGlobalAttention(Bsz, H, N, device=dev, key_block=wl.key_block)
-        layer.load_output_projection(wl.w_o)
-        n_cand = layer.nk - int(wl.keep_k.sum().item())
-        for mname, m in methods:
-            for sp in W.SWEEP_SPARSITIES:
-                c = W.uniform_budget(sp, n_cand)
-                budgets = [c] * H
-                rounds = wl.rounds if m == R.SELECT_DRIFT else 0
+    try:   # printed context only: torch's own dense attention on layer 0
+        import torch.nn.functional as F
+        for _ in range(2):
+            F.scaled_dot_product_attention(wls[0].q, wls[0].k, wls[0].v)
+        flush.fill_(1.0)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        F.scaled_dot_product_attention(wls[0].q, wls[0].k, wls[0].v)
+        b.record()
+        torch.cuda.synchronize()
+        sdpa_ms = a.elapsed_time(b)
+    except Exception:
+        sdpa_ms = None
+    bf16_peak, _, peak_kind = peaks()
+    for mname, m, sp in todo:
+        c = W.uniform_budget(sp, n_cand)
+        budgets = [c] * H
+        tot_ms = tot_fl = kept = 0.0
+        n = 0
+        clocks = ClockSampler(0)
+        clocks.start()
+        for wl in wls:
+            layer.load_output_projection(wl.w_o)
+            rounds = wl.rounds if m == R.SELECT_DRIFT else 0
 
-                def step():
-                    layer.forward(wl.q, wl.k, wl.v, m, budgets, wl.keep_k, wl.dense_q, rounds,
-                                  wl.rho, wl.eps, wl.select_seed)
-                flush.fill_(1.0)
-                step()
-                ts = []
-                for _ in range(2):
-                    flush.fill_(1.0)
-                    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                    a.record()
-                    step()
-                    b.record()
-                    torch.cuda.synchronize()
-                    ts.append(a.elapsed_time(b))
-                if layer.device_error():
-                    raise SystemExit(f"device error {layer.device_error()} in the sweep")
-                fl = kept_tile_flops(layer.kv_idx, layer.kv_cnt, N, wl.key_block)
-                kf = float(layer.kv_cnt.sum().item()) / (Bsz * H * layer.nq * layer.nk)
-                e = acc.setdefault((mname, sp), {"ms": 0.0, "flops": 0.0, "n": 0, "kept": 0.0, "c": c})
-                e["ms"] += sum(ts)
-                e["flops"] += fl * len(ts)
-                e["n"] += len(ts)
-                e["kept"] += kf
-        if li == 0:
-            # printed context only: torch's own dense attention on the same tensors
-            try:
-                import torch.nn.functional as F
-                for _ in range(2):
-                    F.scaled_dot_product_attention(wl.q, wl.k, wl.v)
+            def step():
+                layer.forward(wl.q, wl.k, wl.v, m, budgets, wl.keep_k, wl.dense_q, rounds,
+                              wl.rho, wl.eps, wl.select_seed)
+            flush.fill_(1.0)
+            step()
+            for _ in range(2):
                 flush.fill_(1.0)
                 a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 a.record()
-                F.scaled_dot_product_attention(wl.q, wl.k, wl.v)
+                step()
                 b.record()
                 torch.cuda.synchronize()
-                sdpa_ms = a.elapsed_time(b)
-            except Exception:
-                sdpa_ms = None
-        del wl
-    clk = clocks.stop()
-    bf16_peak, _, peak_kind = peaks()
-    for (mname, sp), e in acc.items():
-        ms = e["ms"] / e["n"]
-        tf = e["flops"] / (e["ms"] * 1e-3) / 1e12
+                tot_ms += a.elapsed_time(b)
+                n += 1
+            if layer.device_error():
+                raise SystemExit(f"device error {layer.device_error()} in the sweep")
+            fl = kept_tile_flops(layer.kv_idx, layer.kv_cnt, N, args.key_block)
+            tot_fl += 2 * fl
+            kept += float(layer.kv_cnt.sum().item()) / (Bsz * H * layer.nq * layer.nk)
+        clk = clocks.stop()
+        tf = tot_fl / (tot_ms * 1e-3) / 1e12
         line = {"metric": METRIC, "sweep": True, "value": round(tf, 3), "unit": "TFLOP/s",
-                "ms_per_layer": round(ms, 4), "layers": args.layers, "steps_per_layer": 2,
+                "ms_per_layer": round(tot_ms / n, 4), "layers": args.layers, "steps_per_layer": 2,
                 "dtype": "bf16", "data": "synthetic (seeded, VGGT-shaped)",
                 "config": {"workload": W.CASES[5].name, "method": mname, "sparsity": sp,
-                           "budget": e["c"], "key_block": args.key_block,
+                           "budget": c, "key_block": args.key_block,
                            "rounds": W.CASES[5].rounds if mname == "drift" else 0,
-                           "kept_tile_fraction": round(e["kept"] / args.layers, 4),
+                           "kept_tile_fraction": round(kept / args.layers, 4),
                            "l2": "flushed before every timed step (256 MiB write)"},
                 "frac_of_bf16_peak": round(tf / bf16_peak, 4), "peak_source": f"{peak_kind} dense bf16 (burst)"}
         if sp == 0.0 and sdpa_ms is not None:
             line["torch_sdpa_dense_ms_layer0"] = round(sdpa_ms, 4)
         if clk:
             line["clocks"] = clk
-        print(json.dumps(line), flush=True)
+        text = json.dumps(line)
+        print(text, flush=True)
+        if args.sweep_out:
+            with open(args.sweep_out, "a") as f:
+                f.write(text + "\n")
 
 
 def main():

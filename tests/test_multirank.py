@@ -141,3 +141,22 @@ def test_reference_arm_runs_on_rank0_only():
     line = json.loads(res[0][0].strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["n_gpus"] == 2
     assert line["value"] > 0 and line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_sweep_resume_skips_recorded_points(tmp_path):
+    """An interrupted sweep resumes at the next point: points already in the JSONL file
+    (same key block and layer count) are skipped; a torn last line is ignored."""
+    import json
+
+    import bench
+    methods = [("mass", 0), ("drift", 1)]
+    sp = (0.0, 0.5, 0.9)
+    out = tmp_path / "sweep.jsonl"
+    assert len(bench.sweep_todo(str(out), methods, sp, 128, 24)) == 6
+    rec = lambda m, s, kb=128, layers=24: json.dumps(
+        {"layers": layers, "config": {"method": m, "sparsity": s, "key_block": kb}})
+    out.write_text("\n".join([rec("mass", 0.0), rec("mass", 0.5), rec("drift", 0.9, kb=64),
+                              rec("drift", 0.0, layers=2)]) + "\n" + '{"layers": 24, "conf')
+    todo = bench.sweep_todo(str(out), methods, sp, 128, 24)
+    assert [(m, s) for m, _, s in todo] == [("mass", 0.9), ("drift", 0.0), ("drift", 0.5),
+                                           ("drift", 0.9)]
