@@ -15,3 +15,17 @@ def pytest_configure(config):
 @pytest.fixture(scope="session")
 def repo_root():
     return ROOT
+
+
+def pytest_sessionfinish(session, exitstatus):
+    """With RESS_PARITY_REPORT=<file>, writes the mask agreement and attention error of
+    every full-layer GPU parity check of the session to that JSON file."""
+    path = os.environ.get("RESS_PARITY_REPORT")
+    if not path:
+        return
+    mod = sys.modules.get("parity")
+    if mod is None or not getattr(mod, "REPORT", None):
+        return
+    import json
+    with open(path, "w") as f:
+        json.dump(mod.REPORT, f, indent=1)

@@ -103,6 +103,11 @@ class OracleLayer:
                                    key_block=self.key_block)
 
 
+# per full-layer parity check: mask agreement and attention error (written out at the end
+# of the session when RESS_PARITY_REPORT names a file; see conftest.py)
+REPORT: list = []
+
+
 def close(got, want, rtol, atol, what):
     got = np.asarray(got, np.float64)
     want = np.asarray(want, np.float64)

@@ -13,8 +13,8 @@ from block_sparse_global_b200 import ress as R
 from block_sparse_global_b200 import workload as W
 from block_sparse_global_b200.pipeline import SparseGlobalAttention
 from oracle import ress_oracle as O
-from parity import (OracleLayer, check_attention, check_drift, check_realized_drift, close,
-                    compare_masks, ensure_built, run_gpu, sample_rows)
+from parity import (REPORT, OracleLayer, check_attention, check_drift, check_realized_drift,
+                    close, compare_masks, ensure_built, run_gpu, sample_rows)
 
 pytestmark = pytest.mark.gpu
 METHODS = {"mass": O.MASS, "drift": O.DRIFT, "random": O.RANDOM}
@@ -51,7 +51,10 @@ def _full_check(wl, method, rows, attn_rows, rounds=None):
     mask = layer.mask.cpu().numpy()
     for (b, h, i) in rows:
         assert sorted(np.nonzero(mask[b, h, i])[0].tolist()) == kept[(b, h, i)]
-    check_attention(layer, orc, attn_rows)
+    worst, rel = check_attention(layer, orc, attn_rows)
+    REPORT.append(dict(workload=wl.case.name, key_block=wl.key_block, method=method,
+                       sparsity=wl.sparsity, **stats, attn_rows=len(attn_rows),
+                       attn_max_abs=worst, attn_rel_l2=rel))
     return layer, orc, stats
 
 
