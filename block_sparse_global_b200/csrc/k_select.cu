@@ -1,9 +1,9 @@
 // Per-(query block, head) key-block selection and the attention launch order.
 //
 // [ReSS] = "ReSS: Residual-Restoring Sparse Attention for 3D Vision Transformers".
-// One warp owns one row (b, h, i); a CTA holds up to 16 rows of the same head so that
+// One warp owns one row (b, h, i); a CTA holds 4, 8 or 16 rows of the same head so that
 // the pooled value tiles streamed through shared memory during restoration (cp.async,
-// double-buffered) serve all of them.  Exact top-k is an MSB-first radix select on
+// three tiles in flight) serve all of them.  Exact top-k is an MSB-first radix select on
 // order-preserving integer keys (8-bit digits, a shared-memory histogram per warp) that
 // finishes by ranking once the threshold bucket holds at most 32 keys; ties go to the
 // lower block index.
@@ -640,9 +640,9 @@ cudaError_t launch_select(const Dims &d, const SelectLaunch &a, cudaStream_t st)
   for (int h = 0; h < d.H; ++h) p.budgets[h] = a.budgets[h];
   const bool restore = a.method == RESS_SELECT_DRIFT && a.rounds > 0;
   const bool state = restore || a.drift != nullptr;
-  // rows per CTA: a power of two (the cooperative gain pass of the restoration rounds
-  // maps 16 rows to lanes); without rounds the rows are independent, and 4 per CTA give
-  // a grid that fills the GPU at small nb
+  // rows per CTA: 4, 8 or 16 (the gain pass of the restoration rounds takes micro-tiles
+  // of 4 rows); without rounds the rows are independent, and 4 per CTA give a grid that
+  // fills the GPU at small nb
   int T = restore ? 16 : 4;
   const bool cdf = a.method == RESS_SELECT_CDF;
   while (T > 4 && select_smem(d.nk, T, restore, state, cdf) > 220 * 1024) T >>= 1;
