@@ -54,6 +54,9 @@ def parse():
                     help="tokens per key block (query blocks are 128); 64 = ReSS Supp. F grid")
     ap.add_argument("--objective", choices=["min", "max-swaps", "max-full"], default="min",
                     help="drift objective: the method, or a drift-maximising control (drift only)")
+    ap.add_argument("--l2-flush", choices=["write", "write+read"], default="write",
+                    help="L2 flush before every timed step: a 256 MiB write, optionally followed "
+                         "by a 256 MiB read that writes the dirty lines back before the step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-groups", type=int, default=4,
@@ -85,6 +88,29 @@ def measured_traffic(workload: str):
     if kv.get("kernel_source_sha256") != sha or kv.get("workload") != workload:
         return None
     return int(kv["dram_bytes_read"]) + int(kv["dram_bytes_write"])
+
+
+class L2Flush:
+    """Evicts the layer's inputs from L2 before a timed step: writes a 256 MiB buffer
+    (twice the 126 MB L2).  With `clean`, it then also reads a second 256 MiB buffer, so
+    that the dirty lines the write left in L2 are written back to HBM here, outside the
+    timed region, instead of during the step's first reads."""
+
+    def __init__(self, dev, clean: bool):
+        import torch
+        self.buf = torch.empty(L2_FLUSH_BYTES // 4, device=dev, dtype=torch.float32)
+        self.clean = clean
+        self.other = torch.ones(L2_FLUSH_BYTES // 4, device=dev, dtype=torch.float32) if clean else None
+
+    def __call__(self):
+        self.buf.fill_(1.0)
+        if self.clean:
+            self.other.sum()
+
+    def describe(self) -> str:
+        return ("flushed before every timed step (256 MiB write, then a 256 MiB read of "
+                "another buffer, so the write's dirty lines leave L2 before the step)"
+                if self.clean else "flushed before every timed step (256 MiB write)")
 
 
 def peaks():
@@ -223,7 +249,7 @@ def run_ours(args):
     keep_k, dense_q = wl.keep_k, wl.dense_q
     layer = SparseGlobalAttention(Bsz, H, N, device=dev, key_block=wl.key_block)
     layer.load_output_projection(wl.w_o)
-    flush = torch.empty(L2_FLUSH_BYTES // 4, device=dev, dtype=torch.float32)
+    flush = L2Flush(dev, args.l2_flush == "write+read")
     stream = torch.cuda.current_stream()
 
     fused = wl.method != R.SELECT_DRIFT   # block map + selection in one kernel
@@ -245,7 +271,7 @@ def run_ours(args):
                                  layer.scale, layer.out, layer.lse, layer.dev_err)
 
     for _ in range(args.warmup):
-        flush.fill_(1.0)
+        flush()
         step()
         attn()
     torch.cuda.synchronize()
@@ -270,7 +296,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     clocks.start()
     for s in range(args.steps):
-        flush.fill_(1.0)
+        flush()
         ev[s][0].record(stream)
         step()
         ev[s][1].record(stream)
@@ -309,7 +335,7 @@ def run_ours(args):
                 continue
             times = []
             for _ in range(5):
-                flush.fill_(1.0)
+                flush()
                 a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 a.record(stream)
                 calls[name]()
@@ -325,7 +351,7 @@ def run_ours(args):
         dense_out = torch.empty_like(layer.out)
         dts = []
         for _ in range(5):
-            flush.fill_(1.0)
+            flush()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
             R.ress_block_sparse_attn(layer.shape, q, k, v, dense_idx, dense_cnt, None, layer.scale, dense_out)
@@ -346,7 +372,7 @@ def run_ours(args):
             layer.make_groups(wl.w_o, groups)
             e2e_ms = []
             for s in range(max(3, args.steps // 2) + 2):
-                flush.fill_(1.0)
+                flush()
                 a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 a.record(stream)
                 layer.forward_host(qh, kh, vh, outh, wl.method, wl.budgets, keep_k, dense_q,
@@ -384,7 +410,7 @@ def run_ours(args):
             "drift_objective": args.objective, "realized_drift_J_mean": float(f"{drift_mean:.6g}"),
             **({"top_p": args.top_p} if wl.method == R.SELECT_CDF else {}),
             "kept_tile_fraction": round(kept_frac, 4), "kept_tile_gflop": round(flops / 1e9, 3),
-            "selection_dtype": "f32", "l2": "flushed before every timed step (256 MiB write)",
+            "selection_dtype": "f32", "l2": flush.describe(),
             "parallelism": f"{world} independent layers, one per GPU" if world > 1 else "single GPU",
         },
         "roofline": {"kernel": "block_sparse_attn", "bound": "tensor", "achieved": round(achieved, 2),
@@ -532,7 +558,7 @@ def run_sweep(args):
     R.load()
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    flush = torch.empty(L2_FLUSH_BYTES // 4, device=dev, dtype=torch.float32)
+    flush = L2Flush(dev, args.l2_flush == "write+read")
     methods = [("mass", R.SELECT_MASS), ("drift", R.SELECT_DRIFT), ("random", R.SELECT_RANDOM)]
     todo = sweep_todo(args.sweep_out, methods, W.SWEEP_SPARSITIES, args.key_block, args.layers)
     if not todo:
@@ -547,7 +573,7 @@ def run_sweep(args):
         import torch.nn.functional as F
         for _ in range(2):
             F.scaled_dot_product_attention(wls[0].q, wls[0].k, wls[0].v)
-        flush.fill_(1.0)
+        flush()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         F.scaled_dot_product_attention(wls[0].q, wls[0].k, wls[0].v)
@@ -571,10 +597,10 @@ def run_sweep(args):
             def step():
                 layer.forward(wl.q, wl.k, wl.v, m, budgets, wl.keep_k, wl.dense_q, rounds,
                               wl.rho, wl.eps, wl.select_seed)
-            flush.fill_(1.0)
+            flush()
             step()
             for _ in range(2):
-                flush.fill_(1.0)
+                flush()
                 a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 a.record()
                 step()
@@ -596,7 +622,7 @@ def run_sweep(args):
                            "budget": c, "key_block": args.key_block,
                            "rounds": W.CASES[5].rounds if mname == "drift" else 0,
                            "kept_tile_fraction": round(kept / args.layers, 4),
-                           "l2": "flushed before every timed step (256 MiB write)"},
+                           "l2": flush.describe()},
                 "frac_of_bf16_peak": round(tf / bf16_peak, 4), "peak_source": f"{peak_kind} dense bf16 (burst)"}
         if sp == 0.0 and sdpa_ms is not None:
             line["torch_sdpa_dense_ms_layer0"] = round(sdpa_ms, 4)

@@ -59,12 +59,12 @@ __global__ void __launch_bounds__(kThreads) head_gram_kernel(const float *__rest
 }
 
 // --------------------------------------------------- mean pooling, [ReSS] §3 step (1)
-// One warp per (tensor, b*h, block).  Lane = (token slot ts = lane/8, 16-byte column
-// group cg = lane%8): a warp-wide load covers 4 consecutive token rows (512 contiguous
-// bytes); 32 such loads cover a 128-token block.  Each lane issues 16 of its loads before
-// it adds any (two halves of the block), so a warp keeps 8 KB in flight; two warps per
-// CTA spread the units over every SM.  Tokens are added in the same order as a plain
-// loop over the block would.
+// One CTA of two warps per (tensor, b*h, block); warp w reads the w-th half of the
+// block's tokens.  Lane = (token slot ts = lane/8, 16-byte column group cg = lane%8): a
+// warp-wide load covers 4 consecutive token rows (512 contiguous bytes), and each lane
+// issues all 16 of its loads before it adds any, so a warp keeps 8 KB in flight and a
+// 128-token block is read by two warps at once.  Within a warp the tokens are added in
+// order; the two halves' sums meet in shared memory and are added (first half + second).
 constexpr int kPoolWarps = 2;
 __global__ void __launch_bounds__(kPoolWarps * 32) pool_kernel(const uint4 *__restrict__ q,
                                                                const uint4 *__restrict__ k,
@@ -73,13 +73,13 @@ __global__ void __launch_bounds__(kPoolWarps * 32) pool_kernel(const uint4 *__re
                                                                float *__restrict__ kp,
                                                                float *__restrict__ vp, long long BH,
                                                                int N, int nq, int nk, int kb) {
-  const int lane = threadIdx.x & 31;
+  __shared__ float part[8][8];  // second half's column sums: [cg][8 columns]
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int cg = lane & 7, ts = lane >> 3;
   // queries are pooled over nq blocks of 128 tokens, keys and values over nk blocks of kb
   const long long q_units = BH * nq, k_units = BH * nk;
   const long long units = q_units + 2 * k_units;
-  for (long long u = (long long)blockIdx.x * kPoolWarps + (threadIdx.x >> 5); u < units;
-       u += (long long)gridDim.x * kPoolWarps) {
+  for (long long u = blockIdx.x; u < units; u += gridDim.x) {
     int which, nbw, bw;
     long long rem;
     if (u < q_units) {
@@ -94,25 +94,23 @@ __global__ void __launch_bounds__(kPoolWarps * 32) pool_kernel(const uint4 *__re
     const uint4 *src = (which == 0 ? q : which == 1 ? k : v) + (size_t)bh * N * 8;
     float *dst = (which == 0 ? qp : which == 1 ? kp : vp) + ((size_t)bh * nbw + j) * kHeadDim;
     const int t0 = j * bw, t1 = min(N, t0 + bw);
+    const int h0 = t0 + warp * (bw / 2), h1 = min(t1, h0 + bw / 2);  // this warp's half
     float acc[8];
 #pragma unroll
     for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+    uint4 w[16];
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      uint4 w[16];
+    for (int it = 0; it < 16; ++it) {
+      const int tok = h0 + ts + 4 * it;
+      w[it] = tok < h1 ? __ldg(src + (size_t)tok * 8 + cg) : make_uint4(0, 0, 0, 0);
+    }
 #pragma unroll
-      for (int it = 0; it < 16; ++it) {
-        const int tok = t0 + ts + 4 * (it + 16 * half);
-        w[it] = tok < t1 ? __ldg(src + (size_t)tok * 8 + cg) : make_uint4(0, 0, 0, 0);
-      }
+    for (int it = 0; it < 16; ++it) {
+      const uint32_t ww[4] = {w[it].x, w[it].y, w[it].z, w[it].w};
 #pragma unroll
-      for (int it = 0; it < 16; ++it) {
-        const uint32_t ww[4] = {w[it].x, w[it].y, w[it].z, w[it].w};
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          acc[2 * c] += __uint_as_float(ww[c] << 16);
-          acc[2 * c + 1] += __uint_as_float(ww[c] & 0xffff0000u);
-        }
+      for (int c = 0; c < 4; ++c) {
+        acc[2 * c] += __uint_as_float(ww[c] << 16);
+        acc[2 * c + 1] += __uint_as_float(ww[c] & 0xffff0000u);
       }
     }
 #pragma unroll
@@ -120,7 +118,14 @@ __global__ void __launch_bounds__(kPoolWarps * 32) pool_kernel(const uint4 *__re
       acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], 8);
       acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], 16);
     }
-    if (ts == 0) {
+    if (warp == 1 && ts == 0) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) part[cg][c] = acc[c];
+    }
+    __syncthreads();
+    if (warp == 0 && ts == 0) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc[c] += part[cg][c];
       const float cnt = (float)(t1 - t0);
       float4 lo = make_float4(__fdiv_rn(acc[0], cnt), __fdiv_rn(acc[1], cnt),
                               __fdiv_rn(acc[2], cnt), __fdiv_rn(acc[3], cnt));
@@ -129,6 +134,7 @@ __global__ void __launch_bounds__(kPoolWarps * 32) pool_kernel(const uint4 *__re
       reinterpret_cast<float4 *>(dst)[2 * cg] = lo;
       reinterpret_cast<float4 *>(dst)[2 * cg + 1] = hi;
     }
+    __syncthreads();  // part[] is free for the next unit
   }
 }
 
@@ -520,8 +526,8 @@ cudaError_t launch_token_gather(const Dims &d, int views, int specials, bool inv
 
 cudaError_t launch_pool(const Dims &d, const void *q, const void *k, const void *v, float *qp,
                         float *kp, float *vp, cudaStream_t st) {
-  const long long units = d.BH() * d.nq + 2 * d.BH() * d.nk;
-  long long blocks = (units + kPoolWarps - 1) / kPoolWarps;
+  const long long units = d.BH() * d.nq + 2 * d.BH() * d.nk;  // one CTA per unit
+  long long blocks = units;
   if (blocks > 148 * 256) blocks = 148 * 256;
   pool_kernel<<<(unsigned)blocks, kPoolWarps * 32, 0, st>>>(
       static_cast<const uint4 *>(q), static_cast<const uint4 *>(k), static_cast<const uint4 *>(v),
