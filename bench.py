@@ -61,6 +61,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-groups", type=int, default=4,
                     help="head groups of the host-buffer call (copy in / kernels / copy out overlap)")
+    ap.add_argument("--e2e-even-groups", action="store_true",
+                    help="equal head groups instead of tapered ones (last group smallest)")
     ap.add_argument("--quick", action="store_true", help="timed loop only (profiling runs)")
     ap.add_argument("--sweep", action="store_true",
                     help="64-view sweep: sparsity {0,25,50,75,90}%% x {mass, drift, random} over "
@@ -369,7 +371,7 @@ def run_ours(args):
             qd, kd, vd = (torch.empty_like(x) for x in (q, k, v))
             # head groups: copies in, kernels and copies out overlap on three streams
             groups = 1 if wl.method == R.SELECT_RANDOM else max(1, min(args.e2e_groups, H))
-            layer.make_groups(wl.w_o, groups)
+            layer.make_groups(wl.w_o, groups, taper=not args.e2e_even_groups)
             e2e_ms = []
             for s in range(max(3, args.steps // 2) + 2):
                 flush()
@@ -384,7 +386,7 @@ def run_ours(args):
                     e2e_ms.append(a.elapsed_time(b))
             em, e2e_flops = reduce_over_ranks(statistics.mean(e2e_ms), flops)
             extra["e2e"] = {"value": round(e2e_flops / (em * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
-                            "ms_per_step": round(em, 4), "head_groups": groups,
+                            "ms_per_step": round(em, 4), "head_groups": [h1 - h0 for h0, h1, _ in layer._groups],
                             "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
                             "d2h_bytes_per_step": layer.out.numel() * layer.out.element_size()}
     bf16_peak, hbm_peak, peak_kind = peaks()

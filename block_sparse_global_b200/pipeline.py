@@ -114,13 +114,35 @@ class SparseGlobalAttention:
         return self.out
 
     # ------------------------------------------------ end to end from host buffers
-    def make_groups(self, w_o: torch.Tensor, groups: int):
-        """Splits the heads into `groups` contiguous ranges for forward_host(): one layer
-        object per range, with its slice of W_O (head h owns columns 64h .. 64h+63)."""
+    @staticmethod
+    def group_sizes(heads: int, groups: int, taper: bool = True) -> list[int]:
+        """Heads per group for forward_host().  The copy in of all groups runs back to
+        back and sets the pace; what is left after it is the last group's kernels and copy
+        out, so with `taper` the sizes fall off linearly (weights groups, groups-1, ..., 1;
+        largest-remainder rounding, at least one head each) and the last group is small."""
+        groups = max(1, min(groups, heads))
+        if not taper:
+            return [heads * (g + 1) // groups - heads * g // groups for g in range(groups)]
+        w = [groups - g for g in range(groups)]
+        extra = heads - groups                     # one head each, then the rest by weight
+        real = [extra * x / sum(w) for x in w]
+        sizes = [1 + int(r) for r in real]
+        order = sorted(range(groups), key=lambda g: (-(real[g] - int(real[g])), g))
+        for g in order[: heads - sum(sizes)]:
+            sizes[g] += 1
+        return sizes
+
+    def make_groups(self, w_o: torch.Tensor, groups: int, taper: bool = True):
+        """Splits the heads into `groups` contiguous ranges for forward_host() (sizes from
+        group_sizes()): one layer object per range, with its slice of W_O (head h owns
+        columns 64h .. 64h+63)."""
         if self.B != 1:
             raise ValueError("forward_host splits heads of one batch element (B = 1)")
-        groups = max(1, min(groups, self.H))
-        bounds = [self.H * g // groups for g in range(groups + 1)]
+        sizes = self.group_sizes(self.H, groups, taper)
+        groups = len(sizes)
+        bounds = [0]
+        for n in sizes:
+            bounds.append(bounds[-1] + n)
         self._groups = []
         for g in range(groups):
             h0, h1 = bounds[g], bounds[g + 1]

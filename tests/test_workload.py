@@ -72,3 +72,21 @@ def test_oracle_layer_runs_on_tiny_case():
         assert all(len(v) == 4 for v in res["kept"].values())
         o, lse = res["attn"][(0, 1, 3)]
         assert o.shape == (128, 64) and np.isfinite(o).all()
+
+
+def test_host_path_head_group_sizes():
+    """Head groups of the host-buffer call: they cover every head once, in contiguous
+    ranges of at least one head; tapered sizes never grow, so the last group is the
+    smallest; the even split differs by at most one."""
+    from block_sparse_global_b200.pipeline import SparseGlobalAttention as S
+    for heads in (1, 2, 3, 7, 16, 24):
+        for groups in (1, 2, 3, 4, 5, 8, 16, 40):
+            for taper in (True, False):
+                sizes = S.group_sizes(heads, groups, taper)
+                assert sum(sizes) == heads and min(sizes) >= 1
+                assert len(sizes) == min(groups, heads)
+                if taper:
+                    assert all(a >= b for a, b in zip(sizes, sizes[1:])), (heads, groups, sizes)
+                else:
+                    assert max(sizes) - min(sizes) <= 1
+    assert S.group_sizes(16, 4) == [6, 5, 3, 2]
