@@ -12,7 +12,7 @@ section / equation:
     [SparseVGGT] "Block-Sparse Global Attention for Efficient Multi-View Geometry
                  Transformers" (abstract page)
 
-Readings of points the pages leave open (each is also listed in the design doc):
+Readings of points the pages leave open:
     pooled map      P = softmax over ALL key blocks of tau * mean(Q_blk) . mean(K_blk),
                     tau = 1/sqrt(d_h): pool first, then softmax ([ReSS] §3 step (1), §4.1).
     special tokens  key blocks flagged always-kept are never candidates; query blocks
