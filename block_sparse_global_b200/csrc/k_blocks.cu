@@ -405,10 +405,20 @@ __global__ void __launch_bounds__(kThreads) drift_prep_kernel(
   __syncthreads();
   const int cnt = rows ? nq : nk;  // vbar has nq rows, the pooled values nk
   const float *src = (rows ? vbar : vp) + (size_t)bh * cnt * kHeadDim;
-  for (int n = blockIdx.x * 32 + warp; n < min(cnt, (int)blockIdx.x * 32 + 32); n += kWarps) {
-    sx[warp][lane] = src[(size_t)n * kHeadDim + lane];
-    sx[warp][lane + 32] = src[(size_t)n * kHeadDim + lane + 32];
+  const int n_end = min(cnt, (int)blockIdx.x * 32 + 32);
+  int n = blockIdx.x * 32 + warp;
+  // this warp's rows n, n + 8, ...: the next row's two values are loaded before the
+  // current row's product, so that the load latency overlaps it
+  float x0 = n < n_end ? src[(size_t)n * kHeadDim + lane] : 0.f;
+  float x1 = n < n_end ? src[(size_t)n * kHeadDim + lane + 32] : 0.f;
+  for (; n < n_end; n += kWarps) {
+    sx[warp][lane] = x0;
+    sx[warp][lane + 32] = x1;
     __syncwarp();
+    if (n + kWarps < n_end) {
+      x0 = src[(size_t)(n + kWarps) * kHeadDim + lane];
+      x1 = src[(size_t)(n + kWarps) * kHeadDim + lane + 32];
+    }
     float y0 = 0.f, y1 = 0.f;
 #pragma unroll 16
     for (int e = 0; e < kHeadDim; ++e) {
@@ -466,7 +476,26 @@ __global__ void __launch_bounds__(kThreads) drift_kernel(
   const int jq = kg * KPM + NV * (ds & 1);
   const float *ch = c + (size_t)bh * nk;
   const bool b2 = ds & 4, b1 = ds & 2, b0 = ds & 1;
+  // P and c of this lane's NV blocks, fetched one tile ahead
+  float pn[NV], cn[NV];
+  auto fetch = [&](int tt) {
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int j = tt * kTileKeys + jq + i;
+      const bool ok = ie < nq && j < nk;
+      pn[i] = ok ? P[orow + j] : 0.f;
+      cn[i] = ok ? ch[j] : 0.f;
+    }
+  };
+  fetch(0);
   tile_stream(tiles, vp + (size_t)bh * nk * kHeadDim, nk, [&](int tt, const float *tile) {
+    float pc[NV], cc[NV];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      pc[i] = pn[i];
+      cc[i] = cn[i];
+    }
+    fetch(tt + 1);
     float acc[4 * KPM];
 #pragma unroll
     for (int kk = 0; kk < KPM; ++kk) {
@@ -500,7 +529,7 @@ __global__ void __launch_bounds__(kThreads) drift_kernel(
 #pragma unroll
       for (int i = 0; i < NV; ++i) {
         const int j = tt * kTileKeys + jq + i;
-        if (j < nk) s[orow + j] = P[orow + j] * sqrtf(fmaxf((ae - 2.f * acc[i]) + ch[j], 0.f));
+        if (j < nk) s[orow + j] = pc[i] * sqrtf(fmaxf((ae - 2.f * acc[i]) + cc[i], 0.f));
       }
     }
   });
