@@ -568,3 +568,26 @@ def test_key_block_64_keep_all_is_dense_attention():
     err = (layer.out.float() - ref).abs().max().item()
     rel = ((layer.out.float() - ref).norm() / ref.norm()).item()
     assert err <= 2e-2 and rel <= 1e-2, (err, rel)
+
+
+def test_maximum_grid_4096_key_blocks():
+    """The largest grid the library accepts: 4096 key blocks per row (one head of 524,288
+    tokens, N(0,1) inputs, no special tokens), drift selection of 40 blocks with two
+    restoration rounds.  At this size the selection runs 4 rows per CTA, the block map 8,
+    and the launch order uses the single-warp scatter; checked against the oracle on
+    sampled rows like the VGGT-shaped layers."""
+    N = 4096 * 128
+    gen = torch.Generator().manual_seed(4096)
+    q, k, v = (torch.randn(1, 1, N, 64, generator=gen).to(torch.bfloat16) for _ in range(3))
+    w_o = torch.randn(64, 64, generator=gen) / 8.0
+    case = W.Case(0, "max-grid-1head-524288tok", heads=1, views=0, seq_len=N, method="drift",
+                  sparsity=1.0 - 40 / 4096, rounds=2, tiny=True)
+    wl = W.Workload(case=case, layer=0, seed=4096, q=q, k=k, v=v, w_o=w_o,
+                    keep_k=torch.zeros(4096, dtype=torch.uint8),
+                    dense_q=torch.zeros(4096, dtype=torch.uint8), budgets=[40],
+                    method=O.DRIFT, rounds=2, select_seed=99, sparsity=case.sparsity)
+    rows = sample_rows(1, 1, 4096, 12, seed=7, always=[(0, 0, 0), (0, 0, 4095)])
+    attn_rows = rows[:6]
+    layer, orc, stats = _full_check(wl, O.DRIFT, rows, attn_rows)
+    cnt = layer.kv_cnt.cpu()
+    assert int(cnt.min()) == 40 and int(cnt.max()) == 40
