@@ -591,3 +591,23 @@ def test_maximum_grid_4096_key_blocks():
     layer, orc, stats = _full_check(wl, O.DRIFT, rows, attn_rows)
     cnt = layer.kv_cnt.cpu()
     assert int(cnt.min()) == 40 and int(cnt.max()) == 40
+
+
+@pytest.mark.parametrize("method", ["mass", "drift"])
+def test_batch_of_two_full_layer(method):
+    """Two batch elements with different seeded inputs through the whole path (pool, block
+    map, drift, selection with restoration, attention): every row against the oracle, so
+    that batch and head indexing (per-head Gram matrix and budget) are both exercised."""
+    a = W.make_workload(2, layer=0, heads=2, views=3, method=method, sparsity=0.6, rounds=3)
+    b = W.make_workload(2, layer=1, heads=2, views=3, method=method, sparsity=0.6, rounds=3)
+    wl = W.Workload(case=a.case, layer=0, seed=a.seed, q=torch.cat([a.q, b.q]),
+                    k=torch.cat([a.k, b.k]), v=torch.cat([a.v, b.v]), w_o=a.w_o,
+                    keep_k=a.keep_k, dense_q=a.dense_q, budgets=[a.budgets[0], a.budgets[1] - 3],
+                    method=a.method, rounds=a.rounds, select_seed=a.select_seed,
+                    sparsity=a.sparsity)
+    rows = _all_rows(2, 2, wl.nb)
+    layer, orc, stats = _full_check(wl, METHODS[method], rows, rows)
+    assert stats["rows"] == len(rows)
+    cnt = layer.kv_cnt.cpu()
+    for bb in range(2):
+        assert int(cnt[bb, 1, 0]) == wl.budgets[1] + int(wl.keep_k.sum())
