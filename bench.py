@@ -10,7 +10,9 @@ sparsity, attention-mass selection.  `--case 3/4` runs the drift workloads inste
 
 value      whole-job effective TFLOP/s over kept tiles (kept-tile FLOPs of all ranks /
            max over ranks of the summed per-step device time); inputs resident in HBM,
-           L2 flushed (256 MiB write) before every timed step.
+           L2 flushed (256 MiB write) before every timed step; the step's kernels are
+           replayed from two CUDA graphs (selection part, attention; `--eager` launches
+           them one by one).
 e2e        the same metric with Q, K, V copied from pinned host memory and the output
            copied back inside every timed step.
 roofline   the attention kernel (dominant): kept-tile FLOPs per launch / its mean CUDA-
@@ -64,6 +66,9 @@ def parse():
     ap.add_argument("--e2e-even-groups", action="store_true",
                     help="equal head groups instead of tapered ones (last group smallest)")
     ap.add_argument("--quick", action="store_true", help="timed loop only (profiling runs)")
+    ap.add_argument("--eager", action="store_true",
+                    help="launch the kernels one by one instead of replaying the step from CUDA "
+                         "graphs (selection part and attention, each captured once)")
     ap.add_argument("--sweep", action="store_true",
                     help="64-view sweep: sparsity {0,25,50,75,90}%% x {mass, drift, random} over "
                          "--layers independent layers, one JSON line per point (not the bench line)")
@@ -291,6 +296,20 @@ def run_ours(args):
     sparse_rows = J[:, :, ~wl.dense_q.bool().to(dev)] if wl.dense_q is not None else J
     drift_mean = float(sparse_rows.mean().item())
 
+    # the timed steps replay CUDA graphs of the same calls (one launch per part instead of
+    # one per kernel); eager launches if asked, or if the capture fails
+    run_step, run_attn = step, attn
+    launch_mode = "eager launches"
+    if not args.eager:
+        try:
+            g_step = SparseGlobalAttention.capture(step)
+            g_attn = SparseGlobalAttention.capture(attn)
+            torch.cuda.synchronize()
+            run_step, run_attn = g_step.replay, g_attn.replay
+            launch_mode = "CUDA graph replay (selection part, attention)"
+        except Exception as exc:   # the step still runs, eagerly
+            torch.cuda.synchronize()
+            launch_mode = f"eager launches (graph capture failed: {type(exc).__name__})"
     clocks = ClockSampler(local)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     if world > 1:
@@ -300,9 +319,9 @@ def run_ours(args):
     for s in range(args.steps):
         flush()
         ev[s][0].record(stream)
-        step()
+        run_step()
         ev[s][1].record(stream)
-        attn()
+        run_attn()
         ev[s][2].record(stream)
     torch.cuda.synchronize()
     if world > 1:
@@ -414,6 +433,7 @@ def run_ours(args):
             "kept_tile_fraction": round(kept_frac, 4), "kept_tile_gflop": round(flops / 1e9, 3),
             "selection_dtype": "f32", "l2": flush.describe(),
             "parallelism": f"{world} independent layers, one per GPU" if world > 1 else "single GPU",
+            "launch": launch_mode,
         },
         "roofline": {"kernel": "block_sparse_attn", "bound": "tensor", "achieved": round(achieved, 2),
                      "peak": bf16_peak, "unit": "TFLOP/s", "frac": round(achieved / bf16_peak, 4),

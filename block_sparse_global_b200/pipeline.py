@@ -113,6 +113,34 @@ class SparseGlobalAttention:
         self.attend(q, k, v, stream)
         return self.out
 
+    # ------------------------------------------------------------- CUDA graphs
+    @staticmethod
+    def capture(fn, warmup: int = 2) -> "torch.cuda.CUDAGraph":
+        """Captures the library calls that `fn()` enqueues on the current stream into a CUDA
+        graph, after `warmup` eager runs on a side stream; `graph.replay()` then launches
+        the same kernels with the same arguments on the current stream.  The library
+        allocates nothing and its launches take only host-side attribute calls, so a layer
+        captures as is; the tensors `fn` uses must keep their addresses (copy new inputs
+        into them before a replay)."""
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for _ in range(warmup):
+                fn()
+        torch.cuda.current_stream().wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            fn()
+        return graph
+
+    def capture_forward(self, q, k, v, method: int, budgets: Sequence[int], keep_k=None,
+                        dense_q=None, rounds: int = 0, rho: float = 0.5, eps: float = 1e-4,
+                        seed: int = 0, top_p: float = 1.0) -> "torch.cuda.CUDAGraph":
+        """forward() on these tensors as one CUDA graph (pool, block map, drift, selection,
+        schedule and attention in one launch of the graph)."""
+        return self.capture(lambda: self.forward(q, k, v, method, budgets, keep_k, dense_q,
+                                                 rounds, rho, eps, seed, top_p=top_p))
+
     # ------------------------------------------------ end to end from host buffers
     @staticmethod
     def group_sizes(heads: int, groups: int, taper: bool = True) -> list[int]:
