@@ -129,7 +129,9 @@ class SparseGlobalAttention:
                 fn()
         torch.cuda.current_stream().wait_stream(side)
         graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
+        # thread-local capture: CUDA calls of other threads (a process group's watchdog,
+        # for one) do not invalidate it; the captured calls themselves allocate nothing
+        with torch.cuda.graph(graph, capture_error_mode="thread_local"):
             fn()
         return graph
 
