@@ -39,9 +39,11 @@ Readings of points the pages leave open:
                     ascending) order are kept until the kept mass, always-kept blocks
                     included, reaches top_p (partial sums in float64), never more than the
                     budget c and never fewer than one candidate when c >= 1.
-Parity status: every function below is pinned by tests/test_oracle_*.py.  The exact
-swap trajectory of the restoration is pinned only through the readings above and the
-brute-force bounds (J_opt <= J_ress <= J_init); the pages print no trajectory.
+Parity status: every function below is pinned by tests/test_oracle_*.py, except one
+part that is parity unpinned: the exact swap trajectory of the restoration rounds
+(select_row with rounds > 0) is pinned only through the readings above and the
+brute-force bounds (J_opt <= J_ress <= J_init, |S| = c, swaps = sum of m_r); the pages
+print no trajectory to check it against.
 """
 from __future__ import annotations
 
