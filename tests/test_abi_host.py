@@ -188,3 +188,38 @@ def test_forced_timeout_diagnostic_validation(lib):
     bad = [FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.c_float(0.0), FAKE]
     assert lib.ress_debug_attn_forced_timeout(shape, *bad, FAKE, i64(1000), None) == INVALID
     assert lib.ress_debug_attn_forced_timeout(None, *args, FAKE, i64(1000), None) == INVALID
+
+
+def test_header_is_plain_c_and_links_from_c(lib, tmp_path):
+    """include/ress.h compiles as strict C99 (no C++ or CUDA headers needed) and a C
+    program links against libress.so and gets host-validation results from it."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    libdir = os.path.dirname(R.LIB_PATH)
+    src = tmp_path / "abi.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include "ress.h"
+int main(void) {
+  ress_shape s = {1, 2, 1024, 64, 128, 0};
+  ress_shape bad = {1, 2, 1024, 32, 128, 0};
+  float *fake = (float *)(unsigned long)0x7F0000000000ul;
+  if (ress_abi_version() != 4) return 2;
+  if (ress_pool_blocks(&s, 0, 0, 0, 0, 0, 0, 0) != RESS_ERR_INVALID_ARG) return 3;
+  if (ress_pool_blocks(&bad, fake, fake, fake, fake, fake, fake, 0) != RESS_ERR_UNSUPPORTED) return 4;
+  printf("%s\n", ress_status_string(RESS_ERR_DEVICE_TIMEOUT));
+  return 0;
+}
+''')
+    exe = tmp_path / "abi"
+    cc = subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                         "-I", os.path.join(root, "include"), str(src), "-L", libdir, "-lress",
+                         f"-Wl,-rpath,{libdir}", "-o", str(exe)], capture_output=True, text=True)
+    assert cc.returncode == 0, cc.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert run.returncode == 0, (run.returncode, run.stdout, run.stderr)
+    assert "TIMEOUT" in run.stdout
