@@ -613,14 +613,14 @@ def test_batch_of_two_full_layer(method):
         assert int(cnt[bb, 1, 0]) == wl.budgets[1] + int(wl.keep_k.sum())
 
 
-@pytest.mark.parametrize("method", ["mass", "drift"])
-def test_cuda_graph_replay_equals_eager(method):
+@pytest.mark.parametrize("method,key_block", [("mass", 128), ("drift", 128), ("drift", 64)])
+def test_cuda_graph_replay_equals_eager(method, key_block):
     """forward() captured into a CUDA graph and replayed gives the eager result bit for
     bit; after new inputs are copied into the captured tensors, a replay computes the new
     layer (again equal to eager)."""
     dev = torch.device("cuda")
     wls = [W.make_workload(2, layer=i, heads=4, views=6, method=method, sparsity=0.75,
-                           rounds=3) for i in (0, 1)]
+                           rounds=3, key_block=key_block) for i in (0, 1)]
     wl = wls[0]
     B, H, N, _ = wl.q.shape
     q, k, v = wl.q.to(dev), wl.k.to(dev), wl.v.to(dev)
@@ -628,13 +628,13 @@ def test_cuda_graph_replay_equals_eager(method):
     args = (METHODS[method], wl.budgets, keep_k, dense_q, wl.rounds, wl.rho, wl.eps, wl.select_seed)
 
     def eager(src):
-        ref = SparseGlobalAttention(B, H, N, device=dev)
+        ref = SparseGlobalAttention(B, H, N, device=dev, key_block=key_block)
         ref.load_output_projection(src.w_o.to(dev))
         ref.forward(src.q.to(dev), src.k.to(dev), src.v.to(dev), *args)
         torch.cuda.synchronize()
         return ref.out.clone(), ref.kv_idx.clone(), ref.kv_cnt.clone()
 
-    layer = SparseGlobalAttention(B, H, N, device=dev)
+    layer = SparseGlobalAttention(B, H, N, device=dev, key_block=key_block)
     layer.load_output_projection(wl.w_o.to(dev))
     graph = layer.capture_forward(q, k, v, *args)
     for src in wls:
