@@ -63,6 +63,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-groups", type=int, default=4,
                     help="head groups of the host-buffer call (copy in / kernels / copy out overlap)")
+    ap.add_argument("--e2e-split", default=None,
+                    help="explicit heads per group of the host-buffer call, e.g. 8,4,2,1,1")
     ap.add_argument("--e2e-even-groups", action="store_true",
                     help="equal head groups instead of tapered ones (last group smallest)")
     ap.add_argument("--quick", action="store_true", help="timed loop only (profiling runs)")
@@ -390,7 +392,9 @@ def run_ours(args):
             qd, kd, vd = (torch.empty_like(x) for x in (q, k, v))
             # head groups: copies in, kernels and copies out overlap on three streams
             groups = 1 if wl.method == R.SELECT_RANDOM else max(1, min(args.e2e_groups, H))
-            layer.make_groups(wl.w_o, groups, taper=not args.e2e_even_groups)
+            split = [int(x) for x in args.e2e_split.split(",")] if args.e2e_split else None
+            layer.make_groups(wl.w_o, groups, taper=not args.e2e_even_groups,
+                              sizes=split if wl.method != R.SELECT_RANDOM else None)
             e2e_ms = []
             for s in range(max(3, args.steps // 2) + 2):
                 flush()

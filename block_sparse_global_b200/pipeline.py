@@ -162,13 +162,20 @@ class SparseGlobalAttention:
             sizes[g] += 1
         return sizes
 
-    def make_groups(self, w_o: torch.Tensor, groups: int, taper: bool = True):
-        """Splits the heads into `groups` contiguous ranges for forward_host() (sizes from
-        group_sizes()): one layer object per range, with its slice of W_O (head h owns
+    def make_groups(self, w_o: torch.Tensor, groups: int, taper: bool = True,
+                    sizes: Optional[Sequence[int]] = None):
+        """Splits the heads into contiguous ranges for forward_host(): `sizes` heads per
+        group if given (positive, summing to the head count), else `groups` groups sized
+        by group_sizes(); one layer object per range, with its slice of W_O (head h owns
         columns 64h .. 64h+63)."""
         if self.B != 1:
             raise ValueError("forward_host splits heads of one batch element (B = 1)")
-        sizes = self.group_sizes(self.H, groups, taper)
+        if sizes is not None:
+            sizes = [int(n) for n in sizes]
+            if min(sizes) < 1 or sum(sizes) != self.H:
+                raise ValueError(f"group sizes {sizes} must be positive and sum to {self.H}")
+        else:
+            sizes = self.group_sizes(self.H, groups, taper)
         groups = len(sizes)
         bounds = [0]
         for n in sizes:
