@@ -367,6 +367,14 @@ def run_ours(args):
                 times.append(a.elapsed_time(b))
             per[name] = round(statistics.median(times), 4)
         extra["kernels_ms"] = per
+        # the HBM-bound step: pooling reads Q, K, V once and writes the fp32 block means
+        _, hbm_peak_gbs, _ = peaks()
+        pool_bytes = 3 * q.numel() * q.element_size() + 4 * Bsz * H * (layer.nq + 2 * layer.nk) * 64
+        if per.get("pool"):
+            gbs = pool_bytes / (per["pool"] * 1e-3) / 1e9
+            extra["hbm_kernels"] = {"pool": {"algorithmic_bytes": pool_bytes, "gbs": round(gbs, 1),
+                                             "frac": round(gbs / hbm_peak_gbs, 4) if hbm_peak_gbs else None,
+                                             "peak_gbs": hbm_peak_gbs}}
         # same-shape dense attention: every query block keeps every key block
         nq, nk = layer.nq, layer.nk
         dense_idx = torch.arange(nk, device=dev, dtype=torch.int32).expand(Bsz, H, nq, nk).contiguous()
@@ -449,6 +457,11 @@ def run_ours(args):
     if clk:
         line["clocks"] = clk
     line.update({k_: v_ for k_, v_ in extra.items() if k_ != "e2e"})
+    if not args.quick:
+        # the exact inputs of this run (seeded generator on the device), for reproducibility
+        import hashlib
+        line["inputs_sha256"] = {n: hashlib.sha256(t.contiguous().view(torch.uint8).cpu().numpy().tobytes()).hexdigest()[:16]
+                                 for n, t in (("q", q), ("k", k), ("v", v))}
     if "e2e" in extra:
         line["e2e"] = extra["e2e"]
     if rank == 0 and not args.no_cpu_baseline and world == 1 and not args.quick:
