@@ -370,11 +370,24 @@ def run_ours(args):
         # the HBM-bound step: pooling reads Q, K, V once and writes the fp32 block means
         _, hbm_peak_gbs, _ = peaks()
         pool_bytes = 3 * q.numel() * q.element_size() + 4 * Bsz * H * (layer.nq + 2 * layer.nk) * 64
-        if per.get("pool"):
-            gbs = pool_bytes / (per["pool"] * 1e-3) / 1e9
-            extra["hbm_kernels"] = {"pool": {"algorithmic_bytes": pool_bytes, "gbs": round(gbs, 1),
-                                             "frac": round(gbs / hbm_peak_gbs, 4) if hbm_peak_gbs else None,
-                                             "peak_gbs": hbm_peak_gbs}}
+        # algorithmic HBM bytes of each block-level step: pooling reads Q, K, V and writes
+        # the fp32 means (HBM-bound); the block map writes P, the drift pass reads P and
+        # writes s, the selection reads P (and s) and writes the kept lists -- those three
+        # are fp32 / latency bound, their GB/s is reported for completeness
+        maps = 4 * Bsz * H * layer.nq * layer.nk
+        lists = 4 * Bsz * H * layer.nq * (layer.nk + 1)
+        bytes_of = {"pool": (pool_bytes, "hbm"),
+                    "block_scores": (maps, "fp32 / latency"),
+                    "drift": (2 * maps, "fp32 / latency"),
+                    "select": ((2 if wl.method == R.SELECT_DRIFT else 1) * maps + lists, "fp32 / latency"),
+                    "scores_select": (lists, "fp32 / latency")}
+        hk = {}
+        for name, (nbytes, bound) in bytes_of.items():
+            if per.get(name):
+                gbs = nbytes / (per[name] * 1e-3) / 1e9
+                hk[name] = {"algorithmic_bytes": nbytes, "gbs": round(gbs, 1), "bound": bound,
+                            "frac": round(gbs / hbm_peak_gbs, 4) if hbm_peak_gbs else None}
+        extra["hbm_kernels"] = dict(hk, peak_gbs=hbm_peak_gbs)
         # same-shape dense attention: every query block keeps every key block
         nq, nk = layer.nq, layer.nk
         dense_idx = torch.arange(nk, device=dev, dtype=torch.int32).expand(Bsz, H, nq, nk).contiguous()
