@@ -39,11 +39,13 @@ Readings of points the pages leave open:
                     ascending) order are kept until the kept mass, always-kept blocks
                     included, reaches top_p (partial sums in float64), never more than the
                     budget c and never fewer than one candidate when c >= 1.
-Parity status: every function below is pinned by tests/test_oracle_*.py, except one
-part that is parity unpinned: the exact swap trajectory of the restoration rounds
-(select_row with rounds > 0) is pinned only through the readings above and the
-brute-force bounds (J_opt <= J_ress <= J_init, |S| = c, swaps = sum of m_r); the pages
-print no trajectory to check it against.
+Parity status: every function below is pinned by tests/test_oracle_*.py.  The
+restoration rounds (select_row with rounds > 0) are pinned move by move: each round's
+restored and dropped blocks are checked against the top-m moves recomputed by a masked
+softmax from the start-of-round drop set, and every J after a round against the
+masked-softmax J of the drop set it leaves; the brute-force bounds (J_opt <= J_ress <=
+J_init, |S| = c, swaps = sum of m_r) hold as well.  What the pages leave open in a round
+(simultaneous choice, rounding of m_r, the K guard) is fixed by the readings above.
 """
 from __future__ import annotations
 
@@ -281,10 +283,10 @@ def select_row(method: int, P_row, cand: Sequence[int], budget: int, *, s_row=No
     gap met on the way, J_init / J_best = Eq. 12 objective of the initial and returned drop
     sets (drift with rounds only), J = realized drift of the returned selection (when M,
     the pooled values and vbar are given), swaps = blocks restored over all rounds,
-    J_trace = J after each round)."""
+    J_trace = J after each round, moves = the blocks each round restored and dropped)."""
     cand = list(cand)
     c = max(0, min(budget, len(cand)))
-    out = dict(margin=math.inf, J_init=None, J_best=None, J=None, swaps=0, J_trace=[])
+    out = dict(margin=math.inf, J_init=None, J_best=None, J=None, swaps=0, J_trace=[], moves=[])
     have_state = M is not None and v_pool_head is not None and vbar_row is not None
 
     def finish(selected, margin, J=None):
@@ -338,6 +340,7 @@ def select_row(method: int, P_row, cand: Sequence[int], budget: int, *, s_row=No
         D = (D - set(restore)) | set(drop)
         S = (S - set(drop)) | set(restore)
         out["swaps"] += len(restore)
+        out["moves"].append(dict(restored=sorted(restore), dropped=sorted(drop)))
         J, G, h = objective(g, K, M, eps, dtype)
         out["J_trace"].append(float(J))
         margin = min(margin, _rel_gap(float(J), float(best_J)))

@@ -301,3 +301,101 @@ def test_cdf_kept_sets_grow_with_the_threshold():
         kept = set(O.cdf_keep(P, list(range(30)), 30, float(tau), 0.0)[0])
         assert prev <= kept
         prev = kept
+
+
+# ------------------------------- the restoration trajectory, move by move ([ReSS] §4.3)
+def _brute_round(logits, Vp, vbar, W, D, S, m, maximise=False):
+    """One restoration round recomputed from its definition, independent of Eqs. 13-16:
+    every candidate move is evaluated by a masked softmax.  From the start-of-round drop
+    set D (reading R7), restoring k changes the objective to J(D - {k}) and dropping k to
+    J(D + {k}); the m restores and the m drops with the largest decrease (largest increase
+    when maximising) are taken, ties to the lower block index.  Returns (restored,
+    dropped, smallest relative gap between the chosen and the next move on either side)."""
+    J0 = _J_masked(logits, Vp, vbar, W, D)
+    sgn = -1.0 if maximise else 1.0
+    up = {k: sgn * (J0 - _J_masked(logits, Vp, vbar, W, D - {k})) for k in D}
+    dn = {k: sgn * (J0 - _J_masked(logits, Vp, vbar, W, D | {k})) for k in S}
+    gap = math.inf
+    picks = []
+    for gains in (up, dn):
+        order = sorted(gains, key=lambda k: (-gains[k], k))
+        if m < len(order):
+            a, b = gains[order[m - 1]], gains[order[m]]
+            gap = min(gap, abs(a - b) / max(abs(a), abs(b), abs(J0), 1e-300))
+        picks.append(sorted(order[:m]))
+    return picks[0], picks[1], gap
+
+
+@pytest.mark.parametrize("sign", [O.MINIMISE, O.MAXIMISE_SWAPS])
+@pytest.mark.parametrize("nk,c,rounds,rho", [(10, 2, 1, 0.5), (10, 4, 1, 0.5), (12, 6, 1, 0.5),
+                                             (11, 4, 1, 1.0), (12, 6, 5, 0.5), (12, 5, 5, 1.0),
+                                             (9, 3, 4, 1.0)])
+def test_restoration_moves_equal_brute_force_moves(nk, c, rounds, rho, sign):
+    """Every round's restored and dropped blocks are the top-m moves of D and of S, both
+    evaluated by a directly recomputed masked softmax from the start-of-round drop set,
+    and every entry of J_trace is the masked-softmax J of the drop set the round leaves
+    (which also checks the Eq. 13 updates of g and K to within rounding).  A top-m taken
+    by the smallest gain, drops chosen after the restores are applied, or drops taken
+    from D instead of S each change some round's moves."""
+    checked = 0
+    for seed in range(10):
+        logits, P, Vp, vbar, W, M, s = _row(500 + 13 * nk + seed, nk=nk)
+        cand = list(range(nk))
+        res = O.select_row(O.DRIFT, P, cand, c, s_row=s, v_pool_head=Vp, vbar_row=vbar, M=M,
+                           rounds=rounds, rho=rho, eps=1e-12, sign=sign, dtype=np.float64)
+        kap = O.rank_key(P, s, 1e-12, np.float64)
+        S = set(sorted(cand, key=lambda j: (-kap[j], j))[:c])
+        D = set(cand) - S
+        assert len(res["moves"]) == rounds and len(res["J_trace"]) == rounds
+        for r in range(rounds):
+            m = O.swap_count(r, c, rho, len(D))
+            restored, dropped, gap = _brute_round(logits, Vp, vbar, W, D, S, m,
+                                                  maximise=sign != O.MINIMISE)
+            if gap < 1e-6:     # a near tie at a cut: either choice is correct
+                break
+            assert res["moves"][r] == dict(restored=restored, dropped=dropped), (seed, r)
+            D = (D - set(restored)) | set(dropped)
+            S = (S - set(dropped)) | set(restored)
+            assert res["J_trace"][r] == pytest.approx(_J_masked(logits, Vp, vbar, W, D),
+                                                      rel=1e-9, abs=1e-18)
+            checked += 1
+    assert checked >= 8 * rounds
+
+
+def test_restoration_move_check_catches_planted_mistakes():
+    """The brute-force move check above fails for the three plausible slips in a round:
+    restores taken by the smallest gain, drops chosen after the restores are applied
+    (sequential instead of from one state), and drops taken from D instead of S.  Each
+    slip is planted in a copy of one round computed here from the oracle's own Eq. 16
+    gains, on the CPU."""
+    caught = {"smallest": 0, "sequential": 0, "from_D": 0}
+    for seed in range(12):
+        logits, P, Vp, vbar, W, M, s = _row(900 + seed, nk=12)
+        cand = list(range(12))
+        kap = O.rank_key(P, s, 1e-12, np.float64)
+        S = set(sorted(cand, key=lambda j: (-kap[j], j))[:5])
+        D = set(cand) - S
+        m = 3
+        want_r, want_d, gap = _brute_round(logits, Vp, vbar, W, D, S, m)
+        if gap < 1e-6:
+            continue
+        s_sq = {j: s[j] ** 2 for j in cand}
+        g, K = O.net_drift(D, P, Vp, vbar, np.float64)
+        J, G, h = O.objective(g, K, M, 1e-12, np.float64)
+        gain, _ = O.swap_gains(D, S, P, s_sq, Vp, vbar, h, G, K, 1e-12, np.float64)
+        top = lambda ks, gn, k: sorted(sorted(ks, key=lambda j: (-gn[j], j))[:k])
+        ok_r, ok_d = top(D, gain, m), top(S, gain, m)
+        assert (ok_r, ok_d) == (want_r, want_d)      # the correct round passes
+        # 1. restores by the smallest gain
+        low = sorted(sorted(D, key=lambda j: (gain[j], j))[:m])
+        caught["smallest"] += low != want_r
+        # 2. sequential: restores applied, gains recomputed, then drops
+        D2 = D - set(ok_r)
+        S2 = S | set(ok_r)
+        g2, K2 = O.net_drift(D2, P, Vp, vbar, np.float64)
+        J2, G2, h2 = O.objective(g2, K2, M, 1e-12, np.float64)
+        gain2, _ = O.swap_gains(D2, S2 - set(ok_r), P, s_sq, Vp, vbar, h2, G2, K2, 1e-12, np.float64)
+        caught["sequential"] += top(S2 - set(ok_r), gain2, m) != want_d
+        # 3. drops taken from D
+        caught["from_D"] += top(D, gain, m) != want_d
+    assert all(v >= 3 for v in caught.values()), caught
