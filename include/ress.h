@@ -230,12 +230,17 @@ ress_status ress_drift_scores(const ress_shape *shape, const float *P, const flo
  * the process exits.  The paper has no counterpart to this call; it exists only for
  * such callers.
  *   Arguments, layouts and results are those of ress_drift_scores, minus the workspace.
- *   Limit: a shape whose ress_drift_workspace_bytes(shape) exceeds 8 MiB (8,388,608
- *   bytes; about 31,700 pooled rows B*H*nb) is rejected with RESS_ERR_UNSUPPORTED before
- *   anything is launched.
+ *   Limit: the scratch this call needs is ress_drift_workspace_bytes(shape) =
+ *   r(B*H*nq*64*4) + r(B*H*nq*4) + r(B*H*nk*4) bytes, each term r(.) rounded up to a
+ *   multiple of 256; a shape for which that exceeds 8 MiB (8,388,608 bytes) is rejected
+ *   with RESS_ERR_UNSUPPORTED before anything is launched.  That is about 31,700 query
+ *   blocks B*H*nq with 128-token key blocks (nk = nq) and about 31,300 with 64-token key
+ *   blocks (nk = 2 nq); ress_drift_workspace_bytes gives the exact figure.
  *   The first call on each device looks up the buffer's device address with a CUDA
  *   runtime call, made with that device current; make this first call before any stream
- *   capture.
+ *   capture.  The address is then kept for the life of the process: calls made after
+ *   cudaDeviceReset (or any other teardown of the device's primary context, after which
+ *   the library's device code is loaded anew) are not supported.
  *   Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
  *   All calls on a device share the one buffer, which keeps the last call's contents
  *   (each call writes every part of it that it later reads, so nothing needs clearing).
