@@ -18,8 +18,9 @@ e2e        the same metric with Q, K, V copied from pinned host memory and the o
            copied back inside every timed step.
 roofline   the attention kernel (dominant): kept-tile FLOPs per launch / its mean CUDA-
            event duration, against the measured dense bf16 tensor-core peak.
-With N > 1 (torchrun) every rank runs its own layer (independent seeds): weak scaling,
-no collective on the data path.
+With N > 1 (torchrun) the heads of the layer are split over the ranks (--shard heads,
+strong scaling) or every rank runs its own layer (--shard layers, weak scaling); either
+way no collective on the data path.
 """
 from __future__ import annotations
 
@@ -71,6 +72,12 @@ def parse():
     ap.add_argument("--e2e-even-groups", action="store_true",
                     help="equal head groups instead of tapered ones (last group smallest)")
     ap.add_argument("--quick", action="store_true", help="timed loop only (profiling runs)")
+    ap.add_argument("--shard", choices=["heads", "layers"], default="heads",
+                    help="with N > 1 GPUs: split the heads of one layer over the ranks (strong "
+                         "scaling), or give every rank its own layer (weak scaling)")
+    ap.add_argument("--unfused", action="store_true",
+                    help="drift: separate block-map, drift-score and selection calls instead of "
+                         "the fused drift-selection kernel")
     ap.add_argument("--eager", action="store_true",
                     help="launch the kernels one by one instead of replaying the step from CUDA "
                          "graphs (selection part and attention, each captured once)")
@@ -261,7 +268,16 @@ def run_ours(args):
         dist.barrier()
     R.load()
 
-    wl = build_case(args, rank)
+    if world > 1 and args.shard == "heads":
+        # one layer, its heads split over the ranks: each rank runs the whole path on its
+        # heads (every step is per head, so nothing crosses ranks on the data path)
+        from block_sparse_global_b200 import workload as W
+        full = build_case(args, 0)
+        h0, h1 = W.head_range(full.q.shape[1], world, rank)
+        wl = W.shard_heads(full, h0, h1)
+        del full
+    else:
+        wl = build_case(args, rank)
     objective = {"min": R.DRIFT_MINIMISE, "max-swaps": R.DRIFT_MAXIMISE_SWAPS,
                  "max-full": R.DRIFT_MAXIMISE_FULL}[args.objective]
     if objective != R.DRIFT_MINIMISE and wl.method != R.SELECT_DRIFT:
@@ -274,18 +290,23 @@ def run_ours(args):
     flush = L2Flush(dev, args.l2_flush == "write+read")
     stream = torch.cuda.current_stream()
 
-    fused = wl.method != R.SELECT_DRIFT   # block map + selection in one kernel
+    drift_method = wl.method == R.SELECT_DRIFT
+    unfused = drift_method and args.unfused   # separate block-map, drift and select calls
 
     def step():
-        if fused:
-            layer.pool(q, k, v)
-            layer.scores_select(wl.method, wl.budgets, keep_k, dense_q, wl.select_seed,
-                                top_p=args.top_p)
-        else:
-            layer.scores(q, k, v)
+        layer.pool(q, k, v)
+        if unfused:
+            R.ress_block_scores(layer.shape, layer.q_pool, layer.k_pool, layer.v_pool, layer.scale,
+                                layer.P, layer.v_bar)
             layer.drift()
             layer.select(wl.method, wl.budgets, keep_k, dense_q, wl.rounds, wl.rho, wl.eps,
                          wl.select_seed, objective=objective)
+        elif drift_method:   # block map, drift score and selection in one kernel
+            layer.drift_select(wl.budgets, keep_k, dense_q, wl.rounds, wl.rho, wl.eps,
+                               objective=objective)
+        else:                # block map and selection in one kernel
+            layer.scores_select(wl.method, wl.budgets, keep_k, dense_q, wl.select_seed,
+                                top_p=args.top_p)
         R.ress_attn_schedule(layer.shape, layer.kv_cnt, layer.order)
 
     def attn():
@@ -304,9 +325,17 @@ def run_ours(args):
     # realized drift J of every row's selection (extra, untimed passes: the block map
     # written out, then the selection with its J output)
     J = torch.zeros(Bsz, H, layer.nq, device=dev)
-    layer.scores(q, k, v)
-    layer.select(wl.method, wl.budgets, keep_k, dense_q, wl.rounds, wl.rho, wl.eps, wl.select_seed,
-                 objective=objective, drift_out=J, top_p=args.top_p)
+    layer.pool(q, k, v)
+    if drift_method and not unfused:
+        layer.drift_select(wl.budgets, keep_k, dense_q, wl.rounds, wl.rho, wl.eps,
+                           objective=objective, drift_out=J)
+    else:
+        R.ress_block_scores(layer.shape, layer.q_pool, layer.k_pool, layer.v_pool, layer.scale,
+                            layer.P, layer.v_bar)
+        if drift_method:
+            layer.drift()
+        layer.select(wl.method, wl.budgets, keep_k, dense_q, wl.rounds, wl.rho, wl.eps,
+                     wl.select_seed, objective=objective, drift_out=J, top_p=args.top_p)
     torch.cuda.synchronize()
     sparse_rows = J[:, :, ~wl.dense_q.bool().to(dev)] if wl.dense_q is not None else J
     drift_mean = float(sparse_rows.mean().item())
@@ -351,9 +380,16 @@ def run_ours(args):
     extra = {}
     if not args.quick:
         # per-kernel breakdown (separate pass, same inputs)
-        names = (["pool", "scores_select", "schedule", "attention"] if fused else
-                 ["pool", "block_scores", "drift", "select", "schedule", "attention"])
+        # the step's own kernels, then (drift) the separate calls the fused kernel replaces
+        if not drift_method:
+            names = ["pool", "scores_select", "schedule", "attention"]
+        elif unfused:
+            names = ["pool", "block_scores", "drift", "select", "schedule", "attention"]
+        else:
+            names = ["pool", "drift_select", "schedule", "attention", "block_scores", "drift", "select"]
         calls = {
+            "drift_select": lambda: layer.drift_select(wl.budgets, keep_k, dense_q, wl.rounds, wl.rho,
+                                                       wl.eps, objective=objective),
             "scores_select": lambda: layer.scores_select(wl.method, wl.budgets, keep_k, dense_q,
                                                          wl.select_seed, top_p=args.top_p),
             "pool": lambda: R.ress_pool_blocks(layer.shape, q, k, v, layer.q_pool, layer.k_pool, layer.v_pool),
@@ -367,8 +403,6 @@ def run_ours(args):
         }
         per = {}
         for name in names:
-            if name == "drift" and wl.method != R.SELECT_DRIFT:
-                continue
             times = []
             for _ in range(5):
                 flush()
@@ -380,6 +414,11 @@ def run_ours(args):
                 times.append(a.elapsed_time(b))
             per[name] = round(statistics.median(times), 4)
         extra["kernels_ms"] = per
+        if drift_method and not unfused:
+            extra["kernels_ms_note"] = ("drift_select = block map + drift score + selection in one "
+                                        "kernel (with its c_j prep launch), the step's path; "
+                                        "block_scores, drift and select are the separate calls it "
+                                        "replaces, timed for comparison")
         # the HBM-bound step: pooling reads Q, K, V once and writes the fp32 block means
         _, hbm_peak_gbs, _ = peaks()
         pool_bytes = 3 * q.numel() * q.element_size() + 4 * Bsz * H * (layer.nq + 2 * layer.nk) * 64
@@ -393,7 +432,8 @@ def run_ours(args):
                     "block_scores": (maps, "fp32 / latency"),
                     "drift": (2 * maps, "fp32 / latency"),
                     "select": ((2 if wl.method == R.SELECT_DRIFT else 1) * maps + lists, "fp32 / latency"),
-                    "scores_select": (lists, "fp32 / latency")}
+                    "scores_select": (lists, "fp32 / latency"),
+                    "drift_select": (lists, "fp32 / latency")}
         hk = {}
         for name, (nbytes, bound) in bytes_of.items():
             if per.get(name):
@@ -409,7 +449,9 @@ def run_ours(args):
         restore_rounds = wl.rounds if wl.method == R.SELECT_DRIFT else 0
         fma_of = {"block_scores": 2 * rows_cols * 64,          # logits and vbar
                   "drift": rows_cols * 64,                      # w_i . V_j
-                  "select": (restore_rounds + 1) * rows_cols * 64 if restore_rounds else 0}
+                  "select": (restore_rounds + 1) * rows_cols * 64 if restore_rounds else 0,
+                  # all three in one kernel
+                  "drift_select": (restore_rounds + 4) * rows_cols * 64 if drift_method else 0}
         fk = {}
         for name, fma in fma_of.items():
             if fma and per.get(name):
@@ -474,7 +516,7 @@ def run_ours(args):
         "warmup": args.warmup,
         "ms_per_step": round(total_ms_max / args.steps, 4),
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": "strong" if world > 1 and args.shard == "heads" else "weak",
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded, VGGT-shaped)",
@@ -486,15 +528,20 @@ def run_ours(args):
             **({"top_p": args.top_p} if wl.method == R.SELECT_CDF else {}),
             "kept_tile_fraction": round(kept_frac, 4), "kept_tile_gflop": round(flops / 1e9, 3),
             "selection_dtype": "f32", "l2": flush.describe(),
-            "parallelism": f"{world} independent layers, one per GPU" if world > 1 else "single GPU",
+            "parallelism": ("single GPU" if world == 1 else
+                            f"heads of one layer split over {world} GPUs ({H} on this rank)"
+                            if args.shard == "heads" else f"{world} independent layers, one per GPU"),
             "launch": launch_mode,
+            "selection_kernel": ("separate block map, drift score and selection calls" if unfused else
+                                 "fused drift selection (block map, drift score, selection)"
+                                 if drift_method else "fused block map + selection"),
         },
         "roofline": {"kernel": "block_sparse_attn", "bound": "tensor", "achieved": round(achieved, 2),
                      "peak": bf16_peak, "unit": "TFLOP/s", "frac": round(achieved / bf16_peak, 4),
                      "peak_source": f"{peak_kind} dense bf16 (burst)",
                      "traffic": measured_traffic(workload_name(wl)), "traffic_unit": "bytes per launch (ncu)",
                      "mean_launch_ms": round(attn_mean, 4)},
-        "gpu_launches": args.steps * layer.kernel_launches(wl.method),
+        "gpu_launches": args.steps * layer.kernel_launches(wl.method, fused=not unfused),
     }
     if clk:
         line["clocks"] = clk

@@ -393,13 +393,14 @@ __global__ void __launch_bounds__(kThreads) block_scores_kernel(
 // c_j = V_j^T M V_j in the workspace.
 __global__ void __launch_bounds__(kThreads) drift_prep_kernel(
     const float *__restrict__ vp, const float *__restrict__ vbar, const float *__restrict__ gram,
-    float *__restrict__ w, float *__restrict__ a, float *__restrict__ c, int H, int nq, int nk) {
+    float *__restrict__ w, float *__restrict__ a, float *__restrict__ c, int H, int nq, int nk,
+    int zbase) {
   __shared__ float sM[kHeadDim][kPad];
   __shared__ float sx[kWarps][kHeadDim];
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const long long bh = blockIdx.y;
   const int h = (int)(bh % H);
-  const bool rows = blockIdx.z == 0;  // 0: vbar rows -> w, a;  1: pooled keys -> c
+  const bool rows = blockIdx.z + zbase == 0;  // 0: vbar rows -> w, a;  1: pooled keys -> c
   for (int idx = t; idx < kHeadDim * kHeadDim; idx += kThreads)
     sM[idx / kHeadDim][idx % kHeadDim] = gram[(size_t)h * kHeadDim * kHeadDim + idx];
   __syncthreads();
@@ -426,7 +427,7 @@ __global__ void __launch_bounds__(kThreads) drift_prep_kernel(
       y0 = fmaf(sM[lane][e], xe, y0);
       y1 = fmaf(sM[lane + 32][e], xe, y1);
     }
-    const float dot = warp_sum(sx[warp][lane] * y0 + sx[warp][lane + 32] * y1);
+    const float dot = warp_sum(quad_lane(sx[warp][lane], y0, sx[warp][lane + 32], y1));
     if (rows) {
       w[((size_t)bh * nq + n) * kHeadDim + lane] = y0;
       w[((size_t)bh * nq + n) * kHeadDim + lane + 32] = y1;
@@ -529,7 +530,7 @@ __global__ void __launch_bounds__(kThreads) drift_kernel(
 #pragma unroll
       for (int i = 0; i < NV; ++i) {
         const int j = tt * kTileKeys + jq + i;
-        if (j < nk) s[orow + j] = pc[i] * sqrtf(fmaxf((ae - 2.f * acc[i]) + cc[i], 0.f));
+        if (j < nk) s[orow + j] = drift_score(pc[i], ae, acc[i], cc[i]);
       }
     }
   });
@@ -618,6 +619,17 @@ size_t drift_workspace_bytes(const Dims &d) {
   return up(nr * kHeadDim * sizeof(float)) + up(nr * sizeof(float)) + up(nc * sizeof(float));
 }
 
+size_t drift_select_workspace_bytes(const Dims &d) {
+  return ((size_t)d.BH() * d.nk * sizeof(float) + 255) & ~(size_t)255;
+}
+
+cudaError_t launch_drift_cdiag(const Dims &d, const float *vp, const float *gram, float *c,
+                               cudaStream_t st) {
+  dim3 g((d.nk + 31) / 32, (unsigned)d.BH(), 1);
+  drift_prep_kernel<<<g, kThreads, 0, st>>>(vp, vp, gram, nullptr, nullptr, c, d.H, d.nq, d.nk, 1);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_drift(const Dims &d, const float *P, const float *vp, const float *vbar,
                          const float *gram, float *s, void *ws, cudaStream_t st) {
   const size_t nr = (size_t)d.BH() * d.nq;
@@ -627,7 +639,7 @@ cudaError_t launch_drift(const Dims &d, const float *P, const float *vp, const f
   float *a = reinterpret_cast<float *>(base + up(nr * kHeadDim * sizeof(float)));
   float *c = reinterpret_cast<float *>(base + up(nr * kHeadDim * sizeof(float)) + up(nr * sizeof(float)));
   dim3 g1((max(d.nq, d.nk) + 31) / 32, (unsigned)d.BH(), 2);
-  drift_prep_kernel<<<g1, kThreads, 0, st>>>(vp, vbar, gram, w, a, c, d.H, d.nq, d.nk);
+  drift_prep_kernel<<<g1, kThreads, 0, st>>>(vp, vbar, gram, w, a, c, d.H, d.nq, d.nk, 0);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   dim3 g2((d.nq + kDriftRows - 1) / kDriftRows, (unsigned)d.BH());

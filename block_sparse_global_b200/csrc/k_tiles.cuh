@@ -74,4 +74,17 @@ RESS_DEV void tile_stream(float *buf, const float *src, int nb, Body body) {
   tile_stream_n<2>(buf, src, nb, body);
 }
 
+// The per-block drift arithmetic, written with explicit rounding (no contraction) so that
+// every kernel that evaluates it -- the separate drift kernels and the fused drift
+// selection -- produces the same bits.
+// Lane part of x . M x (lane holds x[lane], x[lane + 32] and (M x) at the same indices).
+RESS_DEV float quad_lane(float x0, float y0, float x1, float y1) {
+  return __fmaf_rn(x1, y1, __fmul_rn(x0, y0));
+}
+// s_ij = P_ij sqrt(max(a_i - 2 u_ij + c_j, 0)), [ReSS] Eq. 9 with Eq. 5: a_i = vbar^T M vbar,
+// u_ij = (M vbar_i) . V_j, c_j = V_j^T M V_j.
+RESS_DEV float drift_score(float p, float a, float u, float c) {
+  return __fmul_rn(p, sqrtf(fmaxf(__fadd_rn(__fsub_rn(a, __fmul_rn(2.f, u)), c), 0.f)));
+}
+
 }  // namespace ress

@@ -132,6 +132,125 @@ RESS_DEV void warp_top_k(int n, int k, KeyFn key, ValidFn valid, MarkFn mark, ui
   __syncwarp();
 }
 
+// ---------------------------------------------------------------- 16-bit histograms
+// A 256-bin histogram of 16-bit counts packed in 128 words (bin b in half b & 1 of word
+// b >> 1); counts stay below 2^16 because a row has at most 4096 entries.
+RESS_DEV void hist16_add(uint32_t *hist, uint32_t bin) {
+  atomicAdd(&hist[bin >> 1], 1u << ((bin & 1u) * 16u));
+}
+RESS_DEV void hist16_clear(uint32_t *hist) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int w = lane; w < 128; w += 32) hist[w] = 0u;
+}
+
+// warp_top_k for 32-bit keys with the 16-bit histogram, for callers that know how many
+// entries are valid (nvalid) and may have built the first pass's histogram already
+// (first_done: hist holds the counts of every valid key's top byte).  Same result as
+// warp_top_k: the k valid entries with the largest key, ties to the lower index.
+template <typename KeyFn, typename ValidFn, typename MarkFn>
+RESS_DEV void warp_top_k16(int n, int k, int nvalid, KeyFn key, ValidFn valid, MarkFn mark,
+                           uint32_t *hist, int *slot, bool first_done) {
+  const int lane = threadIdx.x & 31;
+  if (k <= 0) return;
+  if (k >= nvalid) {
+    for (int j = lane; j < n; j += 32)
+      if (valid(j)) mark(j);
+    __syncwarp();
+    return;
+  }
+  uint32_t prefix = 0, remaining = (uint32_t)k, bucket = 0;
+  int shift = 32;
+  bool have = first_done;
+#pragma unroll 1
+  while (shift > 0) {
+    const int hi_shift = shift;
+    shift -= 8;
+    if (!have) {
+      hist16_clear(hist);
+      __syncwarp();
+      for (int base = 0; base < n; base += 32) {
+        const int j = base + lane;
+        if (j < n && valid(j)) {
+          const uint32_t kk = key(j);
+          if (hi_shift >= 32 || (kk >> hi_shift) == (prefix >> hi_shift)) hist16_add(hist, (kk >> shift) & 255u);
+        }
+      }
+      __syncwarp();
+    }
+    have = false;
+    // lane l holds bins 255-8l .. 248-8l (highest digits first)
+    uint32_t cnt[8], tot = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const uint32_t b = 255u - (uint32_t)(lane * 8 + q);
+      cnt[q] = (hist[b >> 1] >> ((b & 1u) * 16u)) & 0xFFFFu;
+      tot += cnt[q];
+    }
+    uint32_t incl = tot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const uint32_t excl = incl - tot;
+    const unsigned here = __ballot_sync(0xffffffffu, excl < remaining && remaining <= incl);
+    const int src = __ffs(here) - 1;
+    int digit = 0;
+    uint32_t above = 0, inbin = 0;
+    if (lane == src) {
+      uint32_t acc = excl;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (acc + cnt[q] >= remaining) {
+          digit = 255 - (lane * 8 + q);
+          above = acc;
+          inbin = cnt[q];
+          break;
+        }
+        acc += cnt[q];
+      }
+    }
+    digit = __shfl_sync(0xffffffffu, digit, src);
+    above = __shfl_sync(0xffffffffu, above, src);
+    bucket = __shfl_sync(0xffffffffu, inbin, src);
+    remaining -= above;
+    prefix |= (uint32_t)digit << shift;
+    __syncwarp();
+    if (bucket <= 32) break;
+  }
+  const uint32_t top = prefix >> shift;
+  uint32_t taken = 0;
+  for (int base = 0; base < n; base += 32) {
+    const int j = base + lane;
+    const bool v = j < n && valid(j);
+    const uint32_t kt = v ? (key(j) >> shift) : 0u;
+    if (v && kt > top) mark(j);
+    const bool inb = v && kt == top;
+    const unsigned b = __ballot_sync(0xffffffffu, inb);
+    if (bucket <= 32) {
+      if (inb) slot[taken + __popc(b & lanemask_lt())] = j;
+    } else if (inb && taken + __popc(b & lanemask_lt()) < remaining) {
+      mark(j);
+    }
+    taken += __popc(b);
+  }
+  __syncwarp();
+  if (bucket <= 32) {
+    const bool live = lane < (int)taken;
+    const int j = live ? slot[lane] : 0;
+    const uint32_t kk = live ? key(j) : 0u;
+    uint32_t rank = 0;
+    for (int m = 0; m < (int)taken; ++m) {
+      const int jm = __shfl_sync(0xffffffffu, j, m);
+      const uint32_t km = __shfl_sync(0xffffffffu, kk, m);
+      rank += (km > kk || (km == kk && jm < j)) ? 1u : 0u;
+    }
+    if (live && rank < remaining) mark(j);
+  }
+  __syncwarp();
+}
+
 // Marks the k valid entries with the largest key (ties: lower index) for small k by
 // repeated warp-wide arg-max: every lane keeps the best of its own entries (j = lane,
 // lane + 32, ...), the warp picks the best of the 32, its owner marks it (which makes it

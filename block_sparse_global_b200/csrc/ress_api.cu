@@ -12,7 +12,7 @@ using ress::Dims;
 
 namespace {
 
-constexpr int32_t kAbiVersion = 4;
+constexpr int32_t kAbiVersion = 5;
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -196,7 +196,9 @@ ress_status ress_select_blocks(const ress_shape *shape, const ress_select_params
   a.kv_cnt = kv_cnt;
   a.mask = mask;
   a.dev_err = dev_err;
-  return from_cuda(ress::launch_select(d, a, (cudaStream_t)stream));
+  cudaError_t e = ress::launch_select(d, a, (cudaStream_t)stream);
+  if (e == cudaErrorNotSupported) return RESS_ERR_UNSUPPORTED;
+  return from_cuda(e);
 }
 
 ress_status ress_scores_select(const ress_shape *shape, const ress_select_params *params,
@@ -240,6 +242,74 @@ ress_status ress_scores_select(const ress_shape *shape, const ress_select_params
   a.kv_cnt = kv_cnt;
   a.mask = mask;
   return from_cuda(ress::launch_scores_select(d, a, (cudaStream_t)stream));
+}
+
+size_t ress_drift_select_workspace_bytes(const ress_shape *shape) {
+  Dims d;
+  bool empty;
+  if (check_shape(shape, &d, &empty) != RESS_OK) return 0;
+  return ress::drift_select_workspace_bytes(d);
+}
+
+ress_status ress_drift_select(const ress_shape *shape, const ress_select_params *params,
+                              const float *q_pool, const float *k_pool, const float *v_pool,
+                              const float *gram, float scale, float *P, float *v_bar, float *s,
+                              int32_t *kv_idx, int32_t *kv_cnt, uint8_t *mask, int32_t *dev_err,
+                              void *workspace, size_t workspace_bytes, ress_stream_t stream) {
+  Dims d;
+  bool empty;
+  ress_status st = check_shape(shape, &d, &empty);
+  if (st != RESS_OK) return st;
+  if (params == nullptr || params->budgets == nullptr) return RESS_ERR_INVALID_ARG;
+  if (params->method != RESS_SELECT_DRIFT) return RESS_ERR_INVALID_ARG;
+  for (int h = 0; h < d.H; ++h)
+    if (params->budgets[h] < 0 || params->budgets[h] > d.nk) return RESS_ERR_INVALID_ARG;
+  const int obj = params->objective;
+  if (obj != RESS_DRIFT_MINIMISE && obj != RESS_DRIFT_MAXIMISE_SWAPS && obj != RESS_DRIFT_MAXIMISE_FULL)
+    return RESS_ERR_INVALID_ARG;
+  if (params->rounds < 0 || params->rounds > 64) return RESS_ERR_INVALID_ARG;
+  if (!(params->rho > 0.f) || !(params->rho <= 1.f) || !(params->eps > 0.f)) return RESS_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || scale != scale) return RESS_ERR_INVALID_ARG;
+  if (empty) return RESS_OK;
+  if (!ptr_ok(q_pool) || !ptr_ok(k_pool) || !ptr_ok(v_pool) || !ptr_ok(gram) || !ptr_ok(kv_idx) ||
+      !ptr_ok(kv_cnt) || !ptr_ok(workspace))
+    return RESS_ERR_INVALID_ARG;
+  if (workspace_bytes < ress::drift_select_workspace_bytes(d)) return RESS_ERR_INVALID_ARG;
+  for (const void *o : {(const void *)P, (const void *)v_bar, (const void *)s, (const void *)mask,
+                        (const void *)params->drift})
+    if (o != nullptr && !aligned16(o)) return RESS_ERR_INVALID_ARG;
+  if (dev_err != nullptr && (reinterpret_cast<uintptr_t>(dev_err) & 3u)) return RESS_ERR_INVALID_ARG;
+  ress::DriftSelectLaunch a;
+  a.sel.method = RESS_SELECT_DRIFT;
+  a.sel.rounds = params->rounds;
+  a.sel.rho = params->rho;
+  a.sel.eps = params->eps;
+  a.sel.objective = obj;
+  a.sel.top_p = params->top_p;
+  a.sel.drift = params->drift;
+  a.sel.seed = params->seed;
+  a.sel.budgets = params->budgets;
+  a.sel.keep_k = params->keep_k;
+  a.sel.dense_q = params->dense_q;
+  a.sel.P = nullptr;
+  a.sel.s = nullptr;
+  a.sel.vp = v_pool;
+  a.sel.vbar = nullptr;
+  a.sel.gram = gram;
+  a.sel.kv_idx = kv_idx;
+  a.sel.kv_cnt = kv_cnt;
+  a.sel.mask = mask;
+  a.sel.dev_err = dev_err;
+  a.qp = q_pool;
+  a.kp = k_pool;
+  a.scale = scale;
+  a.P_out = P;
+  a.s_out = s;
+  a.vbar_out = v_bar;
+  a.ws = workspace;
+  cudaError_t e = ress::launch_drift_select(d, a, (cudaStream_t)stream);
+  if (e == cudaErrorNotSupported) return RESS_ERR_UNSUPPORTED;
+  return from_cuda(e);
 }
 
 ress_status ress_attn_schedule(const ress_shape *shape, const int32_t *kv_cnt, int32_t *work_order,

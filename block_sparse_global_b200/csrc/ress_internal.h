@@ -47,6 +47,11 @@ size_t drift_workspace_bytes(const Dims &d);
 cudaError_t launch_drift(const Dims &d, const float *P, const float *vp, const float *vbar,
                          const float *gram, float *s, void *ws, cudaStream_t st);
 
+// Workspace of ress_drift_select: c_j = V_j^T M V_j, [B*H, nk] fp32.
+size_t drift_select_workspace_bytes(const Dims &d);
+cudaError_t launch_drift_cdiag(const Dims &d, const float *vp, const float *gram, float *c,
+                               cudaStream_t st);
+
 struct SelectLaunch {
   int method, rounds, objective;
   float top_p;    // RESS_SELECT_CDF threshold
@@ -61,6 +66,16 @@ struct SelectLaunch {
   int32_t *dev_err;
 };
 cudaError_t launch_select(const Dims &d, const SelectLaunch &a, cudaStream_t st);
+
+// Fused drift selection: block map, drift score and selection in one kernel.
+struct DriftSelectLaunch {
+  SelectLaunch sel;               // method DRIFT; P, s, vbar unused
+  const float *qp, *kp;           // pooled queries and keys (vp, gram in sel)
+  float scale;
+  float *P_out, *s_out, *vbar_out;  // optional
+  void *ws;                       // drift_select_workspace_bytes
+};
+cudaError_t launch_drift_select(const Dims &d, const DriftSelectLaunch &a, cudaStream_t st);
 
 cudaError_t launch_schedule(const Dims &d, const int32_t *kv_cnt, int32_t *order, cudaStream_t st);
 

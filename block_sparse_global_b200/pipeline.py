@@ -37,7 +37,8 @@ class SparseGlobalAttention:
         self.P = torch.empty(B, H, nq, nk, **f32)
         self.v_bar = torch.empty(B, H, nq, 64, **f32)
         self.s = torch.empty(B, H, nq, nk, **f32)
-        self.workspace = torch.empty(max(R.ress_drift_workspace_bytes(self.shape), 16),
+        self.workspace = torch.empty(max(R.ress_drift_workspace_bytes(self.shape),
+                                         R.ress_drift_select_workspace_bytes(self.shape), 16),
                                      device=self.device, dtype=torch.uint8)
         self.kv_idx = torch.empty(B, H, nq, nk, **i32)
         self.kv_cnt = torch.empty(B, H, nq, **i32)
@@ -93,6 +94,20 @@ class SparseGlobalAttention:
                              self.gram if state else None, self.kv_idx, self.kv_cnt, self.mask,
                              self.dev_err, stream)
 
+    def drift_select(self, budgets: Sequence[int], keep_k=None, dense_q=None, rounds: int = 0,
+                     rho: float = 0.5, eps: float = 1e-4, stream=None,
+                     objective: int = R.DRIFT_MINIMISE, drift_out: Optional[torch.Tensor] = None,
+                     write_scores: bool = False):
+        """Block map, drift score and DRIFT selection in one kernel (after pool()); P, v_bar
+        and s are written only with write_scores."""
+        params = R.select_params(R.SELECT_DRIFT, budgets, keep_k, dense_q, rounds, rho, eps, 0,
+                                 objective, drift_out)
+        R.ress_drift_select(self.shape, params, self.q_pool, self.k_pool, self.v_pool, self.gram,
+                            self.scale, self.P if write_scores else None,
+                            self.v_bar if write_scores else None,
+                            self.s if write_scores else None, self.kv_idx, self.kv_cnt,
+                            self.workspace, self.mask, self.dev_err, stream)
+
     def attend(self, q, k, v, stream=None, schedule: bool = True):
         if schedule:
             R.ress_attn_schedule(self.shape, self.kv_cnt, self.order, stream)
@@ -102,14 +117,23 @@ class SparseGlobalAttention:
 
     def forward(self, q, k, v, method: int, budgets: Sequence[int], keep_k=None, dense_q=None,
                 rounds: int = 0, rho: float = 0.5, eps: float = 1e-4, seed: int = 0, stream=None,
-                top_p: float = 1.0):
-        if method == R.SELECT_DRIFT:
-            self.scores(q, k, v, stream)
+                top_p: float = 1.0, write_scores: bool = False, fused: bool = True):
+        """pool -> block map + selection (one kernel: drift_select for DRIFT, scores_select
+        otherwise; with fused=False, DRIFT runs the separate block-map, drift and selection
+        calls) -> schedule -> attention.  write_scores: the fused kernels also write P,
+        v_bar (and s for DRIFT)."""
+        self.pool(q, k, v, stream)
+        if method == R.SELECT_DRIFT and fused:
+            self.drift_select(budgets, keep_k, dense_q, rounds, rho, eps, stream,
+                              write_scores=write_scores)
+        elif method == R.SELECT_DRIFT:
+            R.ress_block_scores(self.shape, self.q_pool, self.k_pool, self.v_pool, self.scale,
+                                self.P, self.v_bar, stream)
             self.drift(stream)
             self.select(method, budgets, keep_k, dense_q, rounds, rho, eps, seed, stream)
-        else:   # the block map and the selection fused in one kernel
-            self.pool(q, k, v, stream)
-            self.scores_select(method, budgets, keep_k, dense_q, seed, stream=stream, top_p=top_p)
+        else:
+            self.scores_select(method, budgets, keep_k, dense_q, seed, write_scores, stream=stream,
+                               top_p=top_p)
         self.attend(q, k, v, stream)
         return self.out
 
@@ -232,11 +256,14 @@ class SparseGlobalAttention:
             main.wait_stream(s)
         return out_host
 
-    def kernel_launches(self, method: int) -> int:
-        """Kernels one forward() launches: drift: pool, scores, drift prep, drift, select,
-        schedule, attention; mass / random: pool, fused scores + select, schedule,
-        attention."""
-        return 7 if method == R.SELECT_DRIFT else 4
+    def kernel_launches(self, method: int, fused: bool = True) -> int:
+        """Kernels one forward() launches: drift fused: pool, drift prep (c_j), fused
+        block map + drift + select, schedule, attention; drift unfused: pool, scores, drift
+        prep, drift, select, schedule, attention; mass / cdf / random: pool, fused scores +
+        select, schedule, attention."""
+        if method == R.SELECT_DRIFT:
+            return 5 if fused else 7
+        return 4
 
     def device_error(self) -> int:
         return int(self.dev_err[0].item())

@@ -65,6 +65,10 @@ _SIGS = {
     "ress_scores_select": (_I32, [ctypes.POINTER(ress_shape), ctypes.POINTER(ress_select_params),
                                   _VP, _VP, _VP, ctypes.c_float, _VP, _VP, _VP, _VP, _VP, _VP,
                                   _VP]),
+    "ress_drift_select_workspace_bytes": (_SZ, [ctypes.POINTER(ress_shape)]),
+    "ress_drift_select": (_I32, [ctypes.POINTER(ress_shape), ctypes.POINTER(ress_select_params),
+                                 _VP, _VP, _VP, _VP, ctypes.c_float, _VP, _VP, _VP, _VP, _VP,
+                                 _VP, _VP, _VP, _SZ, _VP]),
     "ress_attn_schedule": (_I32, [ctypes.POINTER(ress_shape), _VP, _VP, _VP]),
     "ress_block_sparse_attn": (_I32, [ctypes.POINTER(ress_shape), _VP, _VP, _VP, _VP, _VP, _VP,
                                       ctypes.c_float, _VP, _VP, _VP, _VP]),
@@ -215,6 +219,26 @@ def ress_scores_select(shape, params, q_pool, k_pool, v_pool, scale: float, P, v
                                    _stream(stream))
     del keep
     _check("ress_scores_select", st)
+
+
+def ress_drift_select_workspace_bytes(shape) -> int:
+    return int(load().ress_drift_select_workspace_bytes(ctypes.byref(_shape(shape))))
+
+
+def ress_drift_select(shape, params, q_pool, k_pool, v_pool, gram, scale: float, P, v_bar, s,
+                      kv_idx, kv_cnt, workspace: torch.Tensor, mask=None, dev_err=None,
+                      stream=None):
+    """Block map, drift score and DRIFT selection in one kernel; P, v_bar, s may be None."""
+    keep = None
+    if isinstance(params, tuple):
+        params, keep = params
+    st = load().ress_drift_select(ctypes.byref(_shape(shape)), ctypes.byref(params), _ptr(q_pool),
+                                  _ptr(k_pool), _ptr(v_pool), _ptr(gram), float(scale), _ptr(P),
+                                  _ptr(v_bar), _ptr(s), _ptr(kv_idx), _ptr(kv_cnt), _ptr(mask),
+                                  _ptr(dev_err), _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(), _stream(stream))
+    del keep
+    _check("ress_drift_select", st)
 
 
 def ress_token_gather(shape, views: int, specials: int, inverse: bool, src, dst, stream=None):

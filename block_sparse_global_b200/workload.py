@@ -213,6 +213,28 @@ def _vggt_qkv(case: Case, gen: torch.Generator, device) -> tuple:
     return q, k, v, {}
 
 
+def head_range(heads: int, world: int, rank: int) -> tuple[int, int]:
+    """Contiguous heads [h0, h1) of rank `rank` when `heads` heads are split over `world`
+    ranks: sizes differ by at most one, the larger ranges first."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError("rank must lie in [0, world)")
+    base, extra = divmod(heads, world)
+    h0 = rank * base + min(rank, extra)
+    return h0, h0 + base + (1 if rank < extra else 0)
+
+
+def shard_heads(wl: "Workload", h0: int, h1: int) -> "Workload":
+    """The heads [h0, h1) of a workload: Q, K, V and the budgets of those heads and the
+    W_O columns 64 h0 .. 64 h1 - 1 that multiply them (every step of the path is per
+    head, so a shard is computed exactly as inside the whole layer; random-selection keys
+    are drawn per call and so differ from the unsplit layer's)."""
+    import dataclasses
+    return dataclasses.replace(
+        wl, q=wl.q[:, h0:h1].contiguous(), k=wl.k[:, h0:h1].contiguous(),
+        v=wl.v[:, h0:h1].contiguous(), w_o=wl.w_o[:, 64 * h0:64 * h1].contiguous(),
+        budgets=list(wl.budgets[h0:h1]))
+
+
 def make_workload(index: int, layer: int = 0, device="cpu", method: Optional[str] = None,
                   sparsity: Optional[float] = None, rounds: Optional[int] = None,
                   heads: Optional[int] = None, views: Optional[int] = None,

@@ -136,9 +136,9 @@ typedef struct {
                                v_pool, v_bar and gram, and eps > 0.                 */
 } ress_select_params;
 
-/* Version of this ABI (incremented on any incompatible change): 4 (ress_shape gained
- * `key_block`; ress_select_params gained `objective`, `top_p` and `drift`;
- * RESS_SELECT_CDF). */
+/* Version of this ABI (incremented on any change of the exported calls): 5 (version 4:
+ * ress_shape gained `key_block`; ress_select_params gained `objective`, `top_p` and
+ * `drift`; RESS_SELECT_CDF; version 5: ress_drift_select and its workspace query). */
 int32_t ress_abi_version(void);
 
 /* Human-readable name of a status code (static string). */
@@ -285,6 +285,37 @@ ress_status ress_select_blocks(const ress_shape *shape, const ress_select_params
                                const float *v_bar, const float *gram, int32_t *kv_idx,
                                int32_t *kv_cnt, uint8_t *mask, int32_t *dev_err,
                                ress_stream_t stream);
+
+/* Bytes of device workspace that ress_drift_select needs for `shape`. */
+size_t ress_drift_select_workspace_bytes(const ress_shape *shape);
+
+/*
+ * ress_drift_select -- ress_block_scores, ress_drift_scores and ress_select_blocks for the
+ * DRIFT method in one pass per row, the fused per-row selection of [ReSS] §4.3 "Fused
+ * kernel implementation" (Supp. E; Table 1, "w/o fused kernel" row): each row's block map
+ * P (Eq. 1), its drift scores s (Eqs. 5, 6, 9), the rank key (Eq. 7), the top-c and the
+ * `rounds` restoration rounds (Eqs. 10-17) stay on chip, so neither P nor s is written
+ * to memory and read back.  P, v_bar and s are evaluated with the same arithmetic, in the
+ * same order, as the three separate calls, so the kept lists are identical to theirs on
+ * the same pooled inputs, bit for bit.
+ *   params     as for ress_select_blocks; method must be RESS_SELECT_DRIFT (else
+ *              INVALID_ARG); params->drift (realized J per row) may be set.
+ *   q_pool [B,H,nq,64], k_pool and v_pool [B,H,nk,64] fp32 (ress_pool_blocks);
+ *   gram   fp32 [H,64,64] (ress_head_gram);  scale: logit scale, normally 1/sqrt(64).
+ *   P      fp32 [B,H,nq,nk], v_bar fp32 [B,H,nq,64], s fp32 [B,H,nq,nk]: optional
+ *          outputs (NULL = not written), equal to the separate calls' outputs.
+ *   kv_idx, kv_cnt, mask, dev_err: as for ress_select_blocks.
+ *   workspace  DEVICE scratch of at least ress_drift_select_workspace_bytes(shape) bytes
+ *              (c_j = V_j^T M V_j of every key block), owned by the caller, 16-byte
+ *              aligned; overwritten.
+ * Errors as ress_select_blocks; RESS_ERR_UNSUPPORTED if a row's on-chip state does not
+ * fit (never for nk <= 4096).
+ */
+ress_status ress_drift_select(const ress_shape *shape, const ress_select_params *params,
+                              const float *q_pool, const float *k_pool, const float *v_pool,
+                              const float *gram, float scale, float *P, float *v_bar, float *s,
+                              int32_t *kv_idx, int32_t *kv_cnt, uint8_t *mask, int32_t *dev_err,
+                              void *workspace, size_t workspace_bytes, ress_stream_t stream);
 
 /*
  * ress_scores_select -- ress_block_scores and ress_select_blocks in one kernel for the

@@ -43,13 +43,9 @@ def run_gpu(wl, method=None, rounds=None, with_mask=True, seed=None):
     layer = SparseGlobalAttention(b, h, n, device=dev, with_mask=with_mask,
                                   key_block=wl.key_block)
     layer.load_output_projection(wl.w_o.to(dev))
+    # the fused kernels write the block map, vbar and (drift) s as well, for the checks
     layer.forward(q, k, v, method, wl.budgets, wl.keep_k.to(dev), wl.dense_q.to(dev), rounds,
-                  wl.rho, wl.eps, wl.select_seed if seed is None else seed)
-    if method != O.DRIFT:
-        # forward() fuses the block map into the mass / random selection and does not
-        # write P or v_bar; compute them for the checks (identical values: see
-        # test_fused_scores_select_equals_separate_calls)
-        layer.scores(q, k, v)
+                  wl.rho, wl.eps, wl.select_seed if seed is None else seed, write_scores=True)
     torch.cuda.synchronize()
     assert layer.device_error() == 0, f"device error {layer.device_error()}"
     return layer
@@ -204,4 +200,17 @@ def sample_rows(B, H, nb, count, seed, always=()):
     rows = set(always)
     while len(rows) < min(count, B * H * nb):
         rows.add((int(rng.integers(B)), int(rng.integers(H)), int(rng.integers(nb))))
+    return sorted(rows)
+
+
+def rows_per_head(H, nb, per_head, seed, always_i=()):
+    """per_head seeded query blocks of every head (batch 0), always including the query
+    blocks listed in always_i."""
+    rng = np.random.default_rng(seed)
+    rows = set()
+    for h in range(H):
+        pick = set(int(i) for i in always_i)
+        while len(pick) < min(per_head, nb):
+            pick.add(int(rng.integers(nb)))
+        rows |= {(0, h, i) for i in pick}
     return sorted(rows)

@@ -39,7 +39,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert R.ress_abi_version() == 4
+    assert R.ress_abi_version() == 5
     assert R.ress_status_string(0) == "RESS_OK"
     assert R.ress_status_string(5) == "RESS_ERR_DEVICE_TIMEOUT"
     assert R.ress_status_string(99) == "RESS_ERR_UNKNOWN"
@@ -208,7 +208,7 @@ int main(void) {
   ress_shape s = {1, 2, 1024, 64, 128, 0};
   ress_shape bad = {1, 2, 1024, 32, 128, 0};
   float *fake = (float *)(unsigned long)0x7F0000000000ul;
-  if (ress_abi_version() != 4) return 2;
+  if (ress_abi_version() != 5) return 2;
   if (ress_pool_blocks(&s, 0, 0, 0, 0, 0, 0, 0) != RESS_ERR_INVALID_ARG) return 3;
   if (ress_pool_blocks(&bad, fake, fake, fake, fake, fake, fake, 0) != RESS_ERR_UNSUPPORTED) return 4;
   printf("%s\n", ress_status_string(RESS_ERR_DEVICE_TIMEOUT));
@@ -223,3 +223,38 @@ int main(void) {
     run = subprocess.run([str(exe)], capture_output=True, text=True)
     assert run.returncode == 0, (run.returncode, run.stdout, run.stderr)
     assert "TIMEOUT" in run.stdout
+
+
+def test_fused_drift_select_validation(lib):
+    """ress_drift_select rejects bad arguments on the host, before any launch."""
+    shape = ctypes.byref(R.make_shape(1, 2, 1024))   # nq = nk = 8
+    ws = lib.ress_drift_select_workspace_bytes(shape)
+    assert ws >= 2 * 8 * 4 and ws % 256 == 0
+    assert lib.ress_drift_select_workspace_bytes(None) == 0
+
+    def call(method=1, budgets=(4, 4), rounds=2, rho=0.5, eps=1e-4, scale=0.125, qp=FAKE,
+             wsb=None, work=FAKE, P=None, objective=0):
+        p, keep = R.select_params(method, list(budgets), rounds=rounds, rho=rho, eps=eps,
+                                  objective=objective)
+        return lib.ress_drift_select(shape, ctypes.byref(p), qp, FAKE, FAKE, FAKE, scale, P, None,
+                                     None, FAKE, FAKE, None, None, work,
+                                     ws if wsb is None else wsb, None)
+
+    assert call(method=0) == INVALID               # drift selection only
+    assert call(budgets=(4, 9)) == INVALID         # budget > nk
+    assert call(rounds=65) == INVALID
+    assert call(rho=0.0) == INVALID
+    assert call(eps=0.0) == INVALID
+    assert call(scale=0.0) == INVALID
+    assert call(scale=float("nan")) == INVALID
+    assert call(objective=3) == INVALID
+    assert call(qp=None) == INVALID
+    assert call(qp=FAKE + 4) == INVALID            # misaligned
+    assert call(work=None) == INVALID
+    assert call(wsb=ws - 1) == INVALID             # workspace too small
+    assert call(P=FAKE + 8) == INVALID             # misaligned optional output
+    # an empty problem is fine without any pointer
+    empty = ctypes.byref(R.make_shape(0, 2, 1024))
+    p, keep = R.select_params(1, [4, 4], rounds=2)
+    assert lib.ress_drift_select(empty, ctypes.byref(p), *([None] * 4), 0.125, *([None] * 8), 0,
+                                 None) == OK

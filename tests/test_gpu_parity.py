@@ -14,6 +14,7 @@ from block_sparse_global_b200 import workload as W
 from block_sparse_global_b200.pipeline import SparseGlobalAttention
 from oracle import ress_oracle as O
 from parity import (REPORT, OracleLayer, check_attention, check_drift, check_realized_drift,
+                    rows_per_head,
                     close, compare_masks, ensure_built, run_gpu, sample_rows)
 
 pytestmark = pytest.mark.gpu
@@ -165,6 +166,62 @@ def test_fused_scores_select_equals_separate_calls(case, method):
             assert bool((fz.P == -1.0).all()) and bool((fz.v_bar == -1.0).all())
 
 
+def _kv_equal(a, b):
+    """Kept lists equal (counts, and every row's valid prefix of kv_idx)."""
+    assert torch.equal(a.kv_cnt, b.kv_cnt)
+    cnt = a.kv_cnt.unsqueeze(-1)
+    pos = torch.arange(a.nk, device=a.kv_cnt.device).view(1, 1, 1, -1)
+    live = pos < cnt
+    assert torch.equal(torch.where(live, a.kv_idx, 0), torch.where(live, b.kv_idx, 0))
+
+
+@pytest.mark.parametrize("case,kb,heads,sign,rounds", [
+    (2, 128, 4, O.MINIMISE, 4), (2, 128, 4, O.MAXIMISE_FULL, 3), (2, 64, 4, O.MINIMISE, 2),
+    (3, 128, 16, O.MINIMISE, 3), (3, 64, 16, O.MINIMISE, 3), (4, 128, 16, O.MINIMISE, 5),
+    (2, 128, 4, O.MINIMISE, 0)])
+def test_fused_drift_select_equals_separate_calls(case, kb, heads, sign, rounds):
+    """ress_drift_select (block map, drift score and drift selection in one kernel, P and
+    s kept on chip) against ress_block_scores + ress_drift_scores + ress_select_blocks on
+    the same pooled inputs ([ReSS] §4.3 "Fused kernel implementation": the fused round
+    gives the same selection): identical kept lists, masks and realized drift J, and
+    identical P, v_bar and s when it writes them.  Includes the full 100-view layer
+    (1074 key blocks, Dirichlet budgets, R = 5) and the 64-token key-block grid."""
+    ensure_built()
+    kw = dict(device="cuda", key_block=kb, method="drift", rounds=rounds)
+    if case == 2:
+        kw.update(heads=heads, views=6)
+    wl = W.make_workload(case, **kw)
+    B, H, N, _ = wl.q.shape
+    dev = torch.device("cuda")
+    ref = SparseGlobalAttention(B, H, N, device=dev, with_mask=True, key_block=kb)
+    ref.load_output_projection(wl.w_o)
+    ref.scores(wl.q, wl.k, wl.v)
+    ref.drift()
+    J_ref = torch.zeros(B, H, ref.nq, device=dev)
+    ref.select(O.DRIFT, wl.budgets, wl.keep_k, wl.dense_q, rounds, wl.rho, wl.eps, 0,
+               objective=sign, drift_out=J_ref)
+    for write in (False, True):
+        fz = SparseGlobalAttention(B, H, N, device=dev, with_mask=True, key_block=kb)
+        fz.load_output_projection(wl.w_o)
+        fz.pool(wl.q, wl.k, wl.v)
+        for t in (fz.P, fz.v_bar, fz.s):
+            t.fill_(-1.0)
+        J = torch.full((B, H, fz.nq), -1.0, device=dev)
+        fz.drift_select(wl.budgets, wl.keep_k, wl.dense_q, rounds, wl.rho, wl.eps,
+                        objective=sign, drift_out=J, write_scores=write)
+        torch.cuda.synchronize()
+        assert fz.device_error() == 0 and ref.device_error() == 0
+        _kv_equal(fz, ref)
+        assert torch.equal(fz.mask, ref.mask)
+        assert torch.equal(J, J_ref)
+        if write:
+            for name in ("P", "v_bar", "s"):
+                assert torch.equal(getattr(fz, name), getattr(ref, name)), name
+        else:
+            for t in (fz.P, fz.v_bar, fz.s):
+                assert bool((t == -1.0).all())
+
+
 @pytest.mark.parametrize("sign", [O.MINIMISE, O.MAXIMISE_SWAPS, O.MAXIMISE_FULL])
 def test_drift_objective_and_realized_drift_on_oracle_scores(sign):
     """The drift-maximising controls of [ReSS] Fig. 8 (swap only, full) and the realized
@@ -222,19 +279,38 @@ def test_vggt_32view_drift75_r3():
 
 
 def test_vggt_100view_drift90_r5_dirichlet():
+    """The headline layer (100 views, 137,400 tokens, 1074 blocks, drift 90 %, R = 5,
+    Dirichlet budgets) through the fused drift selection: every head, 16 query blocks
+    each (always the first, the last sparse and the last dense query block), attention on
+    3 rows of every head."""
     wl = W.make_workload(4)
     nb = wl.nb
     assert sum(wl.budgets) == 16 * 107
-    rows = sample_rows(1, 16, nb, 48, seed=4, always=[(0, 2, nb - 1)])
-    attn_rows = sample_rows(1, 16, nb, 12, seed=5, always=[(0, 9, nb - 3)])
+    dense = [i for i in range(nb) if int(wl.dense_q[i])]
+    assert dense == list(range(nb - 5, nb))
+    rows = rows_per_head(16, nb, 16, seed=4, always_i=(0, nb - 6, nb - 1))
+    attn_rows = rows_per_head(16, nb, 3, seed=5, always_i=(nb - 6,))
     layer, orc, stats = _full_check(wl, O.DRIFT, rows, attn_rows)
     cnt = layer.kv_cnt.cpu()
     for h in range(16):
         assert int(cnt[0, h, 0]) == min(wl.budgets[h], nb - 5) + 5
+        assert int(cnt[0, h, nb - 1]) == nb
+
+
+def test_vggt_100view_drift90_key_block_64_sampled():
+    """The 100-view layer on the 128 x 64 grid (1074 query blocks, 2147 key blocks):
+    drift with 5 restoration rounds on sampled rows of every head, attention on some."""
+    wl = W.make_workload(4, key_block=64)
+    assert (wl.nq, wl.nk) == (1074, 2147)
+    rows = rows_per_head(16, wl.nq, 4, seed=14, always_i=(wl.nq - 6,))
+    attn_rows = sample_rows(1, 16, wl.nq, 8, seed=15, always=[(0, 4, wl.nq - 1)])
+    _full_check(wl, O.DRIFT, rows, attn_rows)
 
 
 @pytest.mark.parametrize("layer_id,sparsity,method", [(0, 0.0, "mass"), (0, 0.9, "random"),
-                                                       (23, 0.25, "drift"), (11, 0.5, "mass")])
+                                                       (23, 0.25, "drift"), (11, 0.5, "mass"),
+                                                       (5, 0.75, "drift"), (17, 0.9, "drift"),
+                                                       (8, 0.9, "mass")])
 def test_vggt_64view_sweep_points(layer_id, sparsity, method):
     wl = W.make_workload(5, layer=layer_id, method=method, sparsity=sparsity)
     nb = wl.nb

@@ -160,3 +160,60 @@ def test_sweep_resume_skips_recorded_points(tmp_path):
     todo = bench.sweep_todo(str(out), methods, sp, 128, 24)
     assert [(m, s) for m, _, s in todo] == [("mass", 0.9), ("drift", 0.0), ("drift", 0.5),
                                            ("drift", 0.9)]
+
+
+# ------------------------------------------------ heads of one layer split over the ranks
+def test_head_ranges_cover_every_head_once():
+    from block_sparse_global_b200 import workload as W
+    for heads in (1, 2, 5, 16, 17, 128):
+        for world in (1, 2, 3, 4, 8):
+            if world > heads:
+                continue
+            ranges = [W.head_range(heads, world, r) for r in range(world)]
+            covered = [h for a, b in ranges for h in range(a, b)]
+            assert covered == list(range(heads)), (heads, world)
+            sizes = [b - a for a, b in ranges]
+            assert max(sizes) - min(sizes) <= 1 and min(sizes) >= 1
+    with pytest.raises(ValueError):
+        W.head_range(16, 2, 2)
+
+
+def _head_shard_worker(rank: int, world: int, port: int, out) -> None:
+    _init(rank, world, port)
+    try:
+        import numpy as np
+
+        from block_sparse_global_b200 import workload as W
+        from oracle import ress_oracle as O
+        full = W.make_workload(2, heads=5, views=3, method="drift", device="cpu")
+        h0, h1 = W.head_range(5, world, rank)
+        wl = W.shard_heads(full, h0, h1)
+        ok = (torch.equal(wl.q, full.q[:, h0:h1]) and torch.equal(wl.v, full.v[:, h0:h1])
+              and wl.budgets == full.budgets[h0:h1] and torch.equal(wl.keep_k, full.keep_k))
+        # the Gram matrices of the shard's W_O columns are the full layer's, heads h0..h1-1
+        g_shard = O.head_gram(wl.w_o.numpy(), h1 - h0)
+        g_full = O.head_gram(full.w_o.numpy(), 5)[h0:h1]
+        ok = ok and bool(np.array_equal(g_shard, g_full))
+        # every head of the layer is processed by exactly one rank
+        mine = torch.zeros(5, dtype=torch.int64)
+        mine[h0:h1] = 1
+        dist.all_reduce(mine)
+        out.put((rank, ok, mine.tolist()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_head_sharded_layer_two_ranks():
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    out = ctx.Queue()
+    procs = [ctx.Process(target=_head_shard_worker, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = [out.get(timeout=120) for _ in range(2)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, ok, count in res:
+        assert ok, rank
+        assert count == [1, 1, 1, 1, 1]
