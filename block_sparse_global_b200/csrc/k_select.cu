@@ -333,8 +333,10 @@ RESS_DEV void tmem_gather_p(uint32_t tP, const int (&kk)[NB], float (&out)[NB]) 
 
 // gather_drift with P from tensor memory: the same sums in the same order.  The pooled
 // value rows of the next eight blocks are requested before the current eight are summed.
-RESS_DEV void gather_drift_t(const int *list, int n, uint32_t tP, const float *vph, float vb0,
-                             float vb1, float sg, float sk, float &g0, float &g1, float &ksum) {
+// Entries q < n_neg enter with the signs (sg_neg, sk_neg), the rest with (sg, sk).
+RESS_DEV void gather_drift_t(const int *list, int n, int n_neg, uint32_t tP, const float *vph,
+                             float vb0, float vb1, float sg_neg, float sk_neg, float sg, float sk,
+                             float &g0, float &g1, float &ksum) {
   const int lane = threadIdx.x & 31;
   int kk[8];
   float x0[8], x1[8];
@@ -356,9 +358,11 @@ RESS_DEV void gather_drift_t(const int *list, int n, uint32_t tP, const float *v
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
       if (kk[q] >= 0) {
-        g0 = __fadd_rn(g0, sg * __fmul_rn(pk[q], __fsub_rn(vb0, x0[q])));
-        g1 = __fadd_rn(g1, sg * __fmul_rn(pk[q], __fsub_rn(vb1, x1[q])));
-        ksum = __fadd_rn(ksum, sk * pk[q]);
+        const bool neg = q0 + q < n_neg;
+        const float a = neg ? sg_neg : sg, b = neg ? sk_neg : sk;
+        g0 = __fadd_rn(g0, a * __fmul_rn(pk[q], __fsub_rn(vb0, x0[q])));
+        g1 = __fadd_rn(g1, a * __fmul_rn(pk[q], __fsub_rn(vb1, x1[q])));
+        ksum = __fadd_rn(ksum, b * pk[q]);
       }
     }
 #pragma unroll
@@ -370,19 +374,24 @@ RESS_DEV void gather_drift_t(const int *list, int n, uint32_t tP, const float *v
   }
 }
 
-// apply_swaps with P from tensor memory.
-RESS_DEV void apply_swaps_t(uint8_t *flags, int nb, const uint16_t *slist, int ns, uint32_t tP,
-                            const float *vph, float vb0, float vb1, float &g0, float &g1, float &K,
-                            int *list) {
+// Applies the chosen swaps to the net drift g and K (Eq. 13 for restores, its mirror for
+// drops), restores in ascending block order, then drops, with P from tensor memory; flags
+// move to KEPT / DROP.  The restores are found among the ascending list rlist (nr entries)
+// when given, else by a scan of all nb blocks; the drops among the ascending kept list
+// slist.  Both go into one list (this warp's shared memory, room for every block) and
+// are gathered in one pass.
+RESS_DEV void apply_swaps_t(uint8_t *flags, int nb, const uint16_t *rlist, int nr,
+                            const uint16_t *slist, int ns, uint32_t tP, const float *vph, float vb0,
+                            float vb1, float &g0, float &g1, float &K, int *list) {
   const int lane = threadIdx.x & 31;
+  int n = 0, n_restore = 0;
 #pragma unroll 1
   for (int pass = 0; pass < 2; ++pass) {
     const uint8_t target = pass == 0 ? F_TO_KEEP : F_TO_DROP;
-    const int nscan = pass == 0 ? nb : ns;
-    int n = 0;
+    const int nscan = pass == 0 ? (rlist ? nr : nb) : ns;
     for (int c0 = 0; c0 < nscan; c0 += 32) {
       const int q = c0 + lane;
-      const int j = q < nscan ? (pass == 0 ? q : (int)slist[q]) : 0;
+      const int j = q < nscan ? (pass == 0 ? (rlist ? (int)rlist[q] : q) : (int)slist[q]) : 0;
       const bool sel = q < nscan && flags[j] == target;
       const unsigned bal = __ballot_sync(0xffffffffu, sel);
       if (sel) {
@@ -391,11 +400,12 @@ RESS_DEV void apply_swaps_t(uint8_t *flags, int nb, const uint16_t *slist, int n
       }
       n += __popc(bal);
     }
-    __syncwarp();
-    gather_drift_t(list, n, tP, vph, vb0, vb1, pass == 0 ? -1.f : 1.f, pass == 0 ? 1.f : -1.f, g0,
-                   g1, K);
-    __syncwarp();
+    if (pass == 0) n_restore = n;
   }
+  __syncwarp();
+  // restore: g -= P_k e_k, K += P_k; drop: g += P_k e_k, K -= P_k
+  gather_drift_t(list, n, n_restore, tP, vph, vb0, vb1, -1.f, 1.f, 1.f, -1.f, g0, g1, K);
+  __syncwarp();
 }
 
 // Products of the CTA's rows with every pooled vector of one 64-block tile, the scheme of
@@ -784,7 +794,7 @@ __global__ void __launch_bounds__(512) drift_select_kernel(const __grid_constant
       n += __popc(bal);
     }
     __syncwarp();
-    gather_drift_t(list, n, tP, vph, vb0, vb1, 1.f, 1.f, g0, g1, Psum);
+    gather_drift_t(list, n, 0, tP, vph, vb0, vb1, 1.f, 1.f, 1.f, 1.f, g0, g1, Psum);
     __syncwarp();
     if (kept_form) {
       g0 = -g0;
@@ -906,7 +916,8 @@ __global__ void __launch_bounds__(512) drift_select_kernel(const __grid_constant
       warp_top_k16(ns, m, ns, [&](int q) { return gkey(slist[q]); },
                    [&](int q) { return flags[slist[q]] == F_KEPT; },
                    [&](int q) { flags[slist[q]] = F_TO_DROP; }, hist, slot, false);
-      apply_swaps_t(flags, nb, slist, ns, tP, vph, vb0, vb1, g0, g1, K, list);
+      apply_swaps_t(flags, nb, ncand <= 256 ? cand : nullptr, ncand, slist, ns, tP, vph, vb0, vb1,
+                    g0, g1, K, list);
       G = gram_apply(sM, g0, g1, h0, h1);
       J = objective(G, K, p.eps);
       if (maximise ? J > bestJ : J < bestJ) {  // track-best (track-worst when maximising)
