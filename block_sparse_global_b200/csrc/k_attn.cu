@@ -19,7 +19,9 @@
 //   warp 5     tensor-core issuer (one elected thread): S = Q K^T (M=128, N=128, K=64)
 //              and O += P V (M=128, N=64, K=128, A operand read from tensor memory).
 //              Also allocates and frees the 256 tensor-memory columns.
-// Tensor memory: S columns [0,128), P [128,192) as packed bf16 pairs, O [192,256).
+// Tensor memory: S columns [0,128), P [128,192) as packed bf16 pairs, O [192,256).  P of
+// tile j goes in two halves: keys 0..63 as soon as the first four MMAs of O += P V of tile
+// j-1 (which read those columns) are done, keys 64..127 after the whole product.
 // Shared memory: Q 16 KB, K 3 x 16 KB, V 2 x 16 KB, all 128-byte swizzled by TMA.
 //
 // Exponentials: at head_dim 64 the MUFU unit (about 16-21 exp2 per clock per SM) is the
@@ -65,6 +67,7 @@ struct Bars {
   uint64_t s_free;
   uint64_t p_full;
   uint64_t o_done;
+  uint64_t o_half;  // the first four MMAs of O += P V done: P columns [0, 32) free
   uint64_t drain;
   uint64_t never;  // completed by nobody: the diagnostic stall of stall_cycles waits here
   uint32_t tmem_base;
@@ -183,6 +186,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     mbar_init(&bar->s_free, 4);
     mbar_init(&bar->p_full, 4);
     mbar_init(&bar->o_done, 1);
+    mbar_init(&bar->o_half, 1);
     mbar_init(&bar->drain, 1);
     mbar_init(&bar->never, 1);
     bar->abort = 0;
@@ -299,8 +303,10 @@ __global__ void __launch_bounds__(kThreads, 2)
             tc_fence_after();
             const uint64_t dv = smem_desc(sV + sp * kTile);
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
+            for (int k = 0; k < 8; ++k) {
               mma_ts(tmem + kColO, tmem + kColP + 8 * k, dv + 128 * k, kIdescPV, (jp > 0 || k > 0));
+              if (k == 3) mma_commit(&bar->o_half);
+            }
             mma_commit(&bar->o_done);
             mma_commit(&bar->v_empty[sp]);
           }
@@ -397,7 +403,14 @@ __global__ void __launch_bounds__(kThreads, 2)
           }
           acc[c & 3] = fadd2(acc[c & 3], e);
           pk[c] = pack_bf16x2(f2lo(e), f2hi(e));
+          if (c == 31) {
+            // keys 0..63 of P: their columns are free once the first half of the
+            // previous tile's O += P V is done
+            if (j > 0) ok = mbar_wait(&bar->o_half, (j - 1) & 1, abort);
+            if (ok) tmem_st32(trow + kColP, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+          }
         }
+        if (!ok) break;
         const uint64_t a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
         const uint64_t a = fadd2(a01, a23);
         l_run = l_run * alpha + (f2lo(a) + f2hi(a));
@@ -417,7 +430,6 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
           }
         }
-        tmem_st32(trow + kColP, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
         tmem_st32(trow + kColP + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
         tmem_wait_st();
         tc_fence_before();

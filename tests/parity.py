@@ -130,12 +130,13 @@ def check_drift(s_gpu_rows, orc: OracleLayer, rows):
 def compare_masks(gpu_kept, orc_sel, nb, what):
     """Kept lists identical on non-ambiguous rows; >= 99.9 % of mask bits agree."""
     rows = sorted(orc_sel["kept"])
-    diff_bits, amb, mism = 0, 0, []
+    diff_bits, amb, same, mism = 0, 0, 0, []
     for r in rows:
         g = set(gpu_kept[r])
         o = set(orc_sel["kept"][r])
         d = len(g ^ o)
         diff_bits += d
+        same += d == 0
         if orc_sel["margin"][r] <= MARGIN:
             amb += 1
         elif d:
@@ -143,7 +144,8 @@ def compare_masks(gpu_kept, orc_sel, nb, what):
     agree = 1.0 - diff_bits / (len(rows) * nb)
     assert not mism, f"{what}: {len(mism)} non-ambiguous rows differ, e.g. {mism[:3]}"
     assert agree >= 0.999, f"{what}: mask agreement {agree:.5f}"
-    return dict(rows=len(rows), ambiguous=amb, agreement=agree)
+    # rows whose kept list is identical to the oracle's, ambiguous or not
+    return dict(rows=len(rows), ambiguous=amb, identical_rows=same, agreement=agree)
 
 
 def check_realized_drift(J_gpu, gpu_kept, sel, orc: OracleLayer, what):
