@@ -5,7 +5,8 @@
     out = layer.forward(q, k, v, method=..., budgets=[...], keep_k=..., dense_q=...)
 
 Every step runs in the library's kernels; this class only owns the buffers and orders
-the calls on one stream: pool -> block map -> (drift) -> select -> schedule -> attention.
+the calls on one stream: pool -> block map + selection (one kernel; for the drift method
+the block map, drift score and restoration rounds in one kernel) -> schedule -> attention.
 """
 from __future__ import annotations
 
