@@ -359,7 +359,11 @@ __global__ void __launch_bounds__(kThreads) block_scores_kernel(
   for (int q = 0; q < TQ; ++q) a0[q] = a1[q] = 0.f;
   tile_stream(tiles, vp + (size_t)bh * nk * kHeadDim, nk, [&](int tt, const float *tile) {
     const int jn = min(kTileKeys, nk - tt * kTileKeys);
-    for (int kk = warp; kk < jn; kk += kWarps) {
+    // the tile's blocks warp, warp + 8, ... (at most 8), unrolled so that their loads overlap
+#pragma unroll
+    for (int it = 0; it < kTileKeys / kWarps; ++it) {
+      const int kk = warp + kWarps * it;
+      if (kk >= jn) break;
       const float x0 = tile[kk * kTilePad + lane], x1 = tile[kk * kTilePad + lane + 32];
       const float *pc = sl + tt * kTileKeys + kk;
 #pragma unroll

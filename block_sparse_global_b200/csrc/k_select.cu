@@ -609,13 +609,18 @@ __global__ void __launch_bounds__(512) drift_select_kernel(const __grid_constant
         for (int gq = 0; gq < 2; ++gq) {
           if (gq >= ng) break;
           const int g = g0 + 4 * gq;
-          for (int kk = g; kk < jn; kk += 8) {
+          const float *prow0 = reinterpret_cast<const float *>(warp_block(rbase) + 1440) + tt * kTileKeys;
+          const size_t rstride = wbytes / sizeof(float);
+          // the tile's blocks g, g + 8, ... (at most 8), unrolled so that their loads overlap
+#pragma unroll
+          for (int it = 0; it < kTileKeys / 8; ++it) {
+            const int kk = g + 8 * it;
+            if (kk >= jn) break;
             const float x0 = tile[kk * kTilePad + lane], x1 = tile[kk * kTilePad + lane + 32];
-            const int j = tt * kTileKeys + kk;
 #pragma unroll
             for (int q = 0; q < RB; ++q) {
               if (q >= nrows) break;
-              const float pj = reinterpret_cast<const float *>(warp_block(rbase + q) + 1440)[j];
+              const float pj = prow0[q * rstride + kk];
               a0[gq][q] = fmaf(pj, x0, a0[gq][q]);
               a1[gq][q] = fmaf(pj, x1, a1[gq][q]);
             }
@@ -693,20 +698,26 @@ __global__ void __launch_bounds__(512) drift_select_kernel(const __grid_constant
     if (row_live) {
       const float *ch = p.cdiag + (size_t)bh * nb;
       float *srow = p.s_out ? p.s_out + ((size_t)bh * nq + i) * nb : nullptr;
-      for (int c0 = 0; c0 < tc; c0 += 32) {
-        uint32_t pv[32], sv[32];
-        tmem_ld32_sync(tP + c0, pv);
+      for (int c0 = 0; c0 < cu; c0 += 16) {
+        uint32_t pv[16], sv[16];
+        float cj[16];
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
+        for (int q = 0; q < 16; ++q) {
+          const int j = lane + 32 * (c0 + q);
+          cj[q] = c0 + q < cu && j < nb ? ch[j] : 0.f;
+        }
+        tmem_ld16_sync(tP + c0, pv);
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
           const int j = lane + 32 * (c0 + q);
           float sj = 0.f;
-          if (j < nb) {
-            sj = drift_score(__uint_as_float(pv[q]), a_row, gain[j], ch[j]);
+          if (c0 + q < cu && j < nb) {
+            sj = drift_score(__uint_as_float(pv[q]), a_row, gain[j], cj[q]);
             if (srow) srow[j] = sj;
           }
           sv[q] = __float_as_uint(sj);
         }
-        tmem_st32(tS + c0, sv);
+        tmem_st16(tS + c0, sv);
       }
       tmem_wait_st();
     }
