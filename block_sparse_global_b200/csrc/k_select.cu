@@ -892,10 +892,10 @@ __global__ void __launch_bounds__(512) drift_select_kernel(const __grid_constant
       // Restores: the m largest keys of D.  With m <= 32, the m-th largest of the 32 lanes'
       // maxima is a lower bound theta of the m-th largest key (m different entries reach
       // it), so every entry of the answer has a key >= theta; those entries are listed in
-      // ascending order (at most 256, else the whole of D is searched) and the top-m is
-      // taken among them, with the same order and ties as over all of D.
-      uint16_t *cand = reinterpret_cast<uint16_t *>(hist + 128);  // 256 entries
-      int ncand = 1 << 30;
+      // ascending order, behind the kept list S (room for nb - ns >= |D| entries), and the
+      // top-m is taken among them, with the same order and ties as over all of D.
+      uint16_t *cand = slist + ns;
+      int ncand = -1;
       if (m <= 32) {
         uint32_t rank = 0;
         for (int l = 0; l < 32; ++l) {
@@ -905,17 +905,16 @@ __global__ void __launch_bounds__(512) drift_select_kernel(const __grid_constant
         const unsigned at = __ballot_sync(0xffffffffu, rank == (uint32_t)(m - 1));
         const uint32_t theta = __shfl_sync(0xffffffffu, lmax, __ffs(at) - 1);
         ncand = 0;
-        for (int c0 = 0; c0 < nb && ncand <= 256; c0 += 32) {
+        for (int c0 = 0; c0 < nb; c0 += 32) {
           const int j = c0 + lane;
           const bool sel = j < nb && flags[j] == F_DROP && gkey(j) >= theta;
           const unsigned bal = __ballot_sync(0xffffffffu, sel);
-          const int pos = ncand + __popc(bal & lanemask_lt());
-          if (sel && pos < 256) cand[pos] = (uint16_t)j;
+          if (sel) cand[ncand + __popc(bal & lanemask_lt())] = (uint16_t)j;
           ncand += __popc(bal);
         }
         __syncwarp();
       }
-      if (ncand <= 256) {
+      if (ncand >= 0) {
         warp_top_k16(ncand, m, ncand, [&](int q) { return gkey(cand[q]); },
                      [&](int q) { return true; }, [&](int q) { flags[cand[q]] = F_TO_KEEP; },
                      hist, slot, false);
@@ -927,7 +926,7 @@ __global__ void __launch_bounds__(512) drift_select_kernel(const __grid_constant
       warp_top_k16(ns, m, ns, [&](int q) { return gkey(slist[q]); },
                    [&](int q) { return flags[slist[q]] == F_KEPT; },
                    [&](int q) { flags[slist[q]] = F_TO_DROP; }, hist, slot, false);
-      apply_swaps_t(flags, nb, ncand <= 256 ? cand : nullptr, ncand, slist, ns, tP, vph, vb0, vb1,
+      apply_swaps_t(flags, nb, ncand >= 0 ? cand : nullptr, ncand, slist, ns, tP, vph, vb0, vb1,
                     g0, g1, K, list);
       G = gram_apply(sM, g0, g1, h0, h1);
       J = objective(G, K, p.eps);
