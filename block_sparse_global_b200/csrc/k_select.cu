@@ -855,7 +855,7 @@ __global__ void __launch_bounds__(512) drift_select_kernel(const __grid_constant
       auto gkey = [&](int j) { return float_key(maximise ? -gain[j] : gain[j]); };
       // the gains, each lane's largest restore key (for the candidate bound below), and
       // the kept candidates S listed in ascending order for the drop side
-      uint32_t lmax = 0u;
+      uint32_t lmax = 0u, lmax_s = 0u;  // largest restore / drop key of the lane
       int ns = 0;
       for (int c0 = 0; c0 < cu; c0 += 16) {
         uint32_t pv[16], sv[16];
@@ -880,7 +880,9 @@ __global__ void __launch_bounds__(512) drift_select_kernel(const __grid_constant
             }
             const float gj = __fsub_rn(base, __fdiv_rn(__fadd_rn(G, dG), __fmul_rn(Kn, Kn)));
             gain[j] = gj;
-            if (f == F_DROP) lmax = max(lmax, float_key(maximise ? -gj : gj));
+            const uint32_t kj = float_key(maximise ? -gj : gj);
+            if (f == F_DROP) lmax = max(lmax, kj);
+            else lmax_s = max(lmax_s, kj);
           }
           const bool sel = f == F_KEPT;
           const unsigned bal = __ballot_sync(0xffffffffu, sel);
@@ -893,17 +895,22 @@ __global__ void __launch_bounds__(512) drift_select_kernel(const __grid_constant
       // maxima is a lower bound theta of the m-th largest key (m different entries reach
       // it), so every entry of the answer has a key >= theta; those entries are listed in
       // ascending order, behind the kept list S (room for nb - ns >= |D| entries), and the
-      // top-m is taken among them, with the same order and ties as over all of D.
+      // top-m is taken among them, with the same order and ties as over all of D (by a
+      // direct rank when at most 64 are left).  Drops: the same over S, whose entries at
+      // or above its bound go to `slot` when at most 64 of them are.
+      auto mth_lane_max = [&](uint32_t v) {
+        uint32_t rank = 0;
+        for (int l = 0; l < 32; ++l) {
+          const uint32_t o = __shfl_sync(0xffffffffu, v, l);
+          rank += (o > v || (o == v && l < lane)) ? 1u : 0u;
+        }
+        const unsigned at = __ballot_sync(0xffffffffu, rank == (uint32_t)(m - 1));
+        return __shfl_sync(0xffffffffu, v, __ffs(at) - 1);
+      };
       uint16_t *cand = slist + ns;
       int ncand = -1;
       if (m <= 32) {
-        uint32_t rank = 0;
-        for (int l = 0; l < 32; ++l) {
-          const uint32_t o = __shfl_sync(0xffffffffu, lmax, l);
-          rank += (o > lmax || (o == lmax && l < lane)) ? 1u : 0u;
-        }
-        const unsigned at = __ballot_sync(0xffffffffu, rank == (uint32_t)(m - 1));
-        const uint32_t theta = __shfl_sync(0xffffffffu, lmax, __ffs(at) - 1);
+        const uint32_t theta = mth_lane_max(lmax);
         ncand = 0;
         for (int c0 = 0; c0 < nb; c0 += 32) {
           const int j = c0 + lane;
@@ -914,7 +921,10 @@ __global__ void __launch_bounds__(512) drift_select_kernel(const __grid_constant
         }
         __syncwarp();
       }
-      if (ncand >= 0) {
+      if (ncand >= 0 && ncand <= 64) {
+        warp_top_k_small(ncand, m, [&](int q) { return gkey(cand[q]); },
+                         [&](int q) { flags[cand[q]] = F_TO_KEEP; });
+      } else if (ncand >= 0) {
         warp_top_k16(ncand, m, ncand, [&](int q) { return gkey(cand[q]); },
                      [&](int q) { return true; }, [&](int q) { flags[cand[q]] = F_TO_KEEP; },
                      hist, slot, false);
@@ -922,10 +932,29 @@ __global__ void __launch_bounds__(512) drift_select_kernel(const __grid_constant
         warp_top_k16(nb, m, n_drop, gkey, [&](int j) { return flags[j] == F_DROP; },
                      [&](int j) { flags[j] = F_TO_KEEP; }, hist, slot, false);
       }
-      // drops: the m largest keys of S (its c entries, listed above)
-      warp_top_k16(ns, m, ns, [&](int q) { return gkey(slist[q]); },
-                   [&](int q) { return flags[slist[q]] == F_KEPT; },
-                   [&](int q) { flags[slist[q]] = F_TO_DROP; }, hist, slot, false);
+      int nds = -1;
+      uint16_t *dcand = reinterpret_cast<uint16_t *>(slot);  // 64 entries
+      if (m <= 32) {
+        const uint32_t theta = mth_lane_max(lmax_s);
+        nds = 0;
+        for (int c0 = 0; c0 < ns && nds <= 64; c0 += 32) {
+          const int q = c0 + lane;
+          const bool sel = q < ns && gkey(slist[q]) >= theta;
+          const unsigned bal = __ballot_sync(0xffffffffu, sel);
+          const int pos = nds + __popc(bal & lanemask_lt());
+          if (sel && pos < 64) dcand[pos] = slist[q];
+          nds += __popc(bal);
+        }
+        __syncwarp();
+      }
+      if (nds >= 0 && nds <= 64) {
+        warp_top_k_small(nds, m, [&](int q) { return gkey(dcand[q]); },
+                         [&](int q) { flags[dcand[q]] = F_TO_DROP; });
+      } else {
+        warp_top_k16(ns, m, ns, [&](int q) { return gkey(slist[q]); },
+                     [&](int q) { return flags[slist[q]] == F_KEPT; },
+                     [&](int q) { flags[slist[q]] = F_TO_DROP; }, hist, slot, false);
+      }
       apply_swaps_t(flags, nb, ncand >= 0 ? cand : nullptr, ncand, slist, ns, tP, vph, vb0, vb1,
                     g0, g1, K, list);
       G = gram_apply(sM, g0, g1, h0, h1);

@@ -132,6 +132,32 @@ RESS_DEV void warp_top_k(int n, int k, KeyFn key, ValidFn valid, MarkFn mark, ui
   __syncwarp();
 }
 
+// Marks the k entries q < n (n <= 64) with the largest key, ties to the lower q, by a
+// direct rank: lane l holds entries l and l + 32 and counts, over all n entries, those
+// that come before each of its own in (key descending, q ascending) order.  Same result
+// as warp_top_k16 over the same entries, without histogram passes.
+template <typename KeyFn, typename MarkFn>
+RESS_DEV void warp_top_k_small(int n, int k, KeyFn key, MarkFn mark) {
+  const int lane = threadIdx.x & 31;
+  if (k <= 0 || n <= 0) return;
+  const bool v0 = lane < n, v1 = lane + 32 < n;
+  const uint32_t k0 = v0 ? key(lane) : 0u, k1 = v1 ? key(lane + 32) : 0u;
+  uint32_t r0 = 0, r1 = 0;
+  const int top = min(n, 32);
+  for (int l = 0; l < top; ++l) {
+    const uint32_t a = __shfl_sync(0xffffffffu, k0, l);  // entry l
+    const uint32_t b = __shfl_sync(0xffffffffu, k1, l);  // entry l + 32
+    const bool bv = l + 32 < n;
+    r0 += (a > k0 || (a == k0 && l < lane)) ? 1u : 0u;
+    r0 += (bv && b > k0) ? 1u : 0u;  // entry l + 32 comes after entry lane on a tie
+    r1 += (a >= k1) ? 1u : 0u;       // entry l comes before entry lane + 32 on a tie
+    r1 += (bv && (b > k1 || (b == k1 && l < lane))) ? 1u : 0u;
+  }
+  if (v0 && r0 < (uint32_t)k) mark(lane);
+  if (v1 && r1 < (uint32_t)k) mark(lane + 32);
+  __syncwarp();
+}
+
 // ---------------------------------------------------------------- 16-bit histograms
 // A 256-bin histogram of 16-bit counts packed in 128 words (bin b in half b & 1 of word
 // b >> 1); counts stay below 2^16 because a row has at most 4096 entries.
