@@ -60,9 +60,10 @@ def parse():
                     help="tokens per key block (query blocks are 128); 64 = ReSS Supp. F grid")
     ap.add_argument("--objective", choices=["min", "max-swaps", "max-full"], default="min",
                     help="drift objective: the method, or a drift-maximising control (drift only)")
-    ap.add_argument("--l2-flush", choices=["write", "write+read"], default="write",
-                    help="L2 flush before every timed step: a 256 MiB write, optionally followed "
-                         "by a 256 MiB read that writes the dirty lines back before the step")
+    ap.add_argument("--l2-flush", choices=["write", "write+read"], default="write+read",
+                    help="L2 flush before every timed step: a 256 MiB write, then (default) a "
+                         "256 MiB read of another buffer, so that the write's dirty lines go back "
+                         "to HBM before the step instead of during its first kernel's reads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-groups", type=int, default=4,
