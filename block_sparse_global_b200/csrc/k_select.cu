@@ -299,15 +299,8 @@ struct DriftSelectParams {
   int budgets[kMaxHeads];
 };
 
-// Loads 32 consecutive tensor-memory columns of the warp's lane quarter; the values are
+// Loads 16 consecutive tensor-memory columns of the warp's lane quarter; the values are
 // usable once the wait has returned (the empty asm ties every value to the wait).
-RESS_DEV void tmem_ld32_sync(uint32_t taddr, uint32_t (&r)[32]) {
-  tmem_ld32(taddr, r);
-  tmem_wait_ld();
-#pragma unroll
-  for (int q = 0; q < 32; ++q) asm volatile("" : "+r"(r[q]));
-}
-
 RESS_DEV void tmem_ld16_sync(uint32_t taddr, uint32_t (&r)[16]) {
   tmem_ld16(taddr, r);
   tmem_wait_ld();
