@@ -66,12 +66,12 @@ def parse():
                          "to HBM before the step instead of during its first kernel's reads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--e2e-groups", type=int, default=4,
+    ap.add_argument("--e2e-groups", type=int, default=6,
                     help="head groups of the host-buffer call (copy in / kernels / copy out overlap)")
     ap.add_argument("--e2e-split", default=None,
                     help="explicit heads per group of the host-buffer call, e.g. 8,4,2,1,1")
-    ap.add_argument("--e2e-even-groups", action="store_true",
-                    help="equal head groups instead of tapered ones (last group smallest)")
+    ap.add_argument("--e2e-taper", action="store_true",
+                    help="linearly tapered head groups instead of near-equal ones (last group smallest)")
     ap.add_argument("--quick", action="store_true", help="timed loop only (profiling runs)")
     ap.add_argument("--shard", choices=["heads", "layers"], default="heads",
                     help="with N > 1 GPUs: split the heads of one layer over the ranks (strong "
@@ -486,7 +486,7 @@ def run_ours(args):
             # head groups: copies in, kernels and copies out overlap on three streams
             groups = 1 if wl.method == R.SELECT_RANDOM else max(1, min(args.e2e_groups, H))
             split = [int(x) for x in args.e2e_split.split(",")] if args.e2e_split else None
-            layer.make_groups(wl.w_o, groups, taper=not args.e2e_even_groups,
+            layer.make_groups(wl.w_o, groups, taper=args.e2e_taper,
                               sizes=split if wl.method != R.SELECT_RANDOM else None)
             e2e_ms = []
             for s in range(max(3, args.steps // 2) + 2):

@@ -170,14 +170,19 @@ class SparseGlobalAttention:
 
     # ------------------------------------------------ end to end from host buffers
     @staticmethod
-    def group_sizes(heads: int, groups: int, taper: bool = True) -> list[int]:
-        """Heads per group for forward_host().  The copy in of all groups runs back to
-        back and sets the pace; what is left after it is the last group's kernels and copy
-        out, so with `taper` the sizes fall off linearly (weights groups, groups-1, ..., 1;
-        largest-remainder rounding, at least one head each) and the last group is small."""
+    def group_sizes(heads: int, groups: int, taper: bool = False) -> list[int]:
+        """Heads per group for forward_host().  The copies in run back to back and set the
+        pace as long as each group's kernels end before the next group's copy in does;
+        after the last copy in, the last group's kernels and copy out are what is left.
+        By default the groups are near-equal, the larger ones first (sizes differ by at
+        most one and never grow), which keeps the kernels behind the copies when they take
+        nearly as long per head (the 100-view layer); with `taper` the sizes fall off
+        linearly (weights groups, groups-1, ..., 1; largest-remainder rounding, at least
+        one head each), which suits layers whose kernels are much shorter than their
+        copies."""
         groups = max(1, min(groups, heads))
         if not taper:
-            return [heads * (g + 1) // groups - heads * g // groups for g in range(groups)]
+            return [heads // groups + (1 if g < heads % groups else 0) for g in range(groups)]
         w = [groups - g for g in range(groups)]
         extra = heads - groups                     # one head each, then the rest by weight
         real = [extra * x / sum(w) for x in w]
@@ -187,7 +192,7 @@ class SparseGlobalAttention:
             sizes[g] += 1
         return sizes
 
-    def make_groups(self, w_o: torch.Tensor, groups: int, taper: bool = True,
+    def make_groups(self, w_o: torch.Tensor, groups: int, taper: bool = False,
                     sizes: Optional[Sequence[int]] = None):
         """Splits the heads into contiguous ranges for forward_host(): `sizes` heads per
         group if given (positive, summing to the head count), else `groups` groups sized

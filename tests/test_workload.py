@@ -76,8 +76,8 @@ def test_oracle_layer_runs_on_tiny_case():
 
 def test_host_path_head_group_sizes():
     """Head groups of the host-buffer call: they cover every head once, in contiguous
-    ranges of at least one head; tapered sizes never grow, so the last group is the
-    smallest; the even split differs by at most one."""
+    ranges of at least one head; sizes never grow, so the last group is the smallest;
+    the default (near-equal) split differs by at most one."""
     from block_sparse_global_b200.pipeline import SparseGlobalAttention as S
     for heads in (1, 2, 3, 7, 16, 24):
         for groups in (1, 2, 3, 4, 5, 8, 16, 40):
@@ -85,8 +85,8 @@ def test_host_path_head_group_sizes():
                 sizes = S.group_sizes(heads, groups, taper)
                 assert sum(sizes) == heads and min(sizes) >= 1
                 assert len(sizes) == min(groups, heads)
-                if taper:
-                    assert all(a >= b for a, b in zip(sizes, sizes[1:])), (heads, groups, sizes)
-                else:
+                assert all(a >= b for a, b in zip(sizes, sizes[1:])), (heads, groups, sizes)
+                if not taper:
                     assert max(sizes) - min(sizes) <= 1
-    assert S.group_sizes(16, 4) == [6, 5, 3, 2]
+    assert S.group_sizes(16, 4, taper=True) == [6, 5, 3, 2]
+    assert S.group_sizes(16, 6) == [3, 3, 3, 3, 2, 2]
