@@ -10,7 +10,9 @@
 //                        in tensor memory.  Its fused form also computes P, vbar and s.
 // Exact top-k is an MSB-first radix select on order-preserving integer keys (8-bit
 // digits, a shared-memory histogram per warp) that finishes by ranking once the
-// threshold bucket holds at most 32 keys; ties go to the lower block index.
+// threshold bucket holds at most 32 keys; ties go to the lower block index.  The
+// restoration rounds' top-m (m <= 32) first keeps only the entries at or above the m-th
+// largest of the 32 lanes' maxima and ranks them directly when at most 64 remain.
 #include "k_tiles.cuh"
 #include "k_topk.cuh"
 #include "ress_common.cuh"
