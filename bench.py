@@ -487,7 +487,8 @@ def run_ours(args):
             groups = 1 if wl.method == R.SELECT_RANDOM else max(1, min(args.e2e_groups, H))
             split = [int(x) for x in args.e2e_split.split(",")] if args.e2e_split else None
             layer.make_groups(wl.w_o, groups, taper=args.e2e_taper,
-                              sizes=split if wl.method != R.SELECT_RANDOM else None)
+                              sizes=split if wl.method != R.SELECT_RANDOM else None,
+                              budgets=wl.budgets if wl.method != R.SELECT_RANDOM else None)
             e2e_ms = []
             for s in range(max(3, args.steps // 2) + 2):
                 flush()
@@ -502,7 +503,7 @@ def run_ours(args):
                     e2e_ms.append(a.elapsed_time(b))
             em, e2e_flops = reduce_over_ranks(statistics.mean(e2e_ms), flops)
             extra["e2e"] = {"value": round(e2e_flops / (em * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
-                            "ms_per_step": round(em, 4), "head_groups": [h1 - h0 for h0, h1, _ in layer._groups],
+                            "ms_per_step": round(em, 4), "head_groups": [heads for _, _, _, heads in layer._groups],
                             "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
                             "d2h_bytes_per_step": layer.out.numel() * layer.out.element_size()}
     bf16_peak, hbm_peak, peak_kind = peaks()

@@ -192,12 +192,39 @@ class SparseGlobalAttention:
             sizes[g] += 1
         return sizes
 
+    @staticmethod
+    def plan_head_order(budgets: Sequence[int], sizes: Sequence[int]) -> list[int]:
+        """Heads in processing order for groups of the given sizes.  The kernels of a
+        head take time roughly in proportion to its budget (its kept blocks), the copies
+        the same time for every head, so the cheapest heads go to the last group (what is
+        left after the last copy in), and the other heads are spread over the other groups
+        largest first, each to the group with the least work per head so far, so that no
+        group's kernels outlast the next group's copy in.  Heads keep ascending order
+        within a group."""
+        H, G = len(budgets), len(sizes)
+        if G <= 1:
+            return list(range(H))
+        cost = [int(b) + 16 for b in budgets]  # kept candidates + always-kept / fixed work
+        asc = sorted(range(H), key=lambda h: (cost[h], h))
+        last = asc[:sizes[-1]]
+        rest = sorted(asc[sizes[-1]:], key=lambda h: (-cost[h], h))
+        members: list[list[int]] = [[] for _ in range(G - 1)]
+        load = [0] * (G - 1)
+        for h in rest:
+            g = min((g for g in range(G - 1) if len(members[g]) < sizes[g]),
+                    key=lambda g: (load[g] / sizes[g], g))
+            members[g].append(h)
+            load[g] += cost[h]
+        return [h for m in members for h in sorted(m)] + sorted(last)
+
     def make_groups(self, w_o: torch.Tensor, groups: int, taper: bool = False,
-                    sizes: Optional[Sequence[int]] = None):
-        """Splits the heads into contiguous ranges for forward_host(): `sizes` heads per
-        group if given (positive, summing to the head count), else `groups` groups sized
-        by group_sizes(); one layer object per range, with its slice of W_O (head h owns
-        columns 64h .. 64h+63)."""
+                    sizes: Optional[Sequence[int]] = None,
+                    budgets: Optional[Sequence[int]] = None):
+        """Splits the heads into groups for forward_host(): `sizes` heads per group if
+        given (positive, summing to the head count), else `groups` groups sized by
+        group_sizes().  With `budgets`, the heads are assigned by plan_head_order();
+        without, group g takes the next contiguous range.  One layer object per group,
+        with the W_O columns of its heads (head h owns columns 64h .. 64h+63)."""
         if self.B != 1:
             raise ValueError("forward_host splits heads of one batch element (B = 1)")
         if sizes is not None:
@@ -206,17 +233,19 @@ class SparseGlobalAttention:
                 raise ValueError(f"group sizes {sizes} must be positive and sum to {self.H}")
         else:
             sizes = self.group_sizes(self.H, groups, taper)
-        groups = len(sizes)
-        bounds = [0]
-        for n in sizes:
-            bounds.append(bounds[-1] + n)
+        order = self.plan_head_order(budgets, sizes) if budgets is not None else list(range(self.H))
+        if sorted(order) != list(range(self.H)):
+            raise ValueError("the head order must be a permutation of the heads")
+        self._order = order
         self._groups = []
-        for g in range(groups):
-            h0, h1 = bounds[g], bounds[g + 1]
-            sub = SparseGlobalAttention(1, h1 - h0, self.N, device=self.device,
-                                        key_block=self.key_block)
-            sub.load_output_projection(w_o[:, 64 * h0:64 * h1])
-            self._groups.append((h0, h1, sub))
+        s0 = 0
+        for n in sizes:
+            heads = order[s0:s0 + n]
+            sub = SparseGlobalAttention(1, n, self.N, device=self.device, key_block=self.key_block)
+            cols = torch.cat([torch.arange(64 * h, 64 * h + 64, device=w_o.device) for h in heads])
+            sub.load_output_projection(w_o[:, cols])
+            self._groups.append((s0, s0 + n, sub, heads))
+            s0 += n
         self._streams = [torch.cuda.Stream(self.device) for _ in range(3)]
         return self._groups
 
@@ -227,37 +256,54 @@ class SparseGlobalAttention:
         """The layer end to end from pinned host tensors [1,H,N,64] bf16 to the pinned host
         output.  Heads are processed in the groups of make_groups(): the copy in of group
         g+1, the kernels of group g and the copy out of group g-1 run on three streams and
-        overlap.  RANDOM selection runs as one group (its keys depend on the head index
+        overlap.  The device staging tensors hold the heads in processing order (slot s
+        holds head make_groups' order[s]); contiguous runs of heads are copied in one piece.
+        RANDOM selection runs as one group in head order (its keys depend on the head index
         within the call).  The caller's current stream waits for the whole layer.
         q_dev, k_dev, v_dev: optional device staging tensors of the same shape."""
         groups = getattr(self, "_groups", None)
         if not groups:
             raise RuntimeError("call make_groups() first")
-        if method == R.SELECT_RANDOM and len(groups) > 1:
-            raise ValueError("random selection runs as one group")
+        if method == R.SELECT_RANDOM and (len(groups) > 1 or self._order != list(range(self.H))):
+            raise ValueError("random selection runs as one group in head order")
         q_dev = torch.empty_like(q_host, device=self.device) if q_dev is None else q_dev
         k_dev = torch.empty_like(k_host, device=self.device) if k_dev is None else k_dev
         v_dev = torch.empty_like(v_host, device=self.device) if v_dev is None else v_dev
+        budgets = list(budgets)
         s_in, s_cmp, s_out = self._streams
         main = torch.cuda.current_stream(self.device)
         for s in (s_in, s_cmp, s_out):
             s.wait_stream(main)
-        for (h0, h1, sub) in groups:
+
+        def runs(s0, heads):
+            # (first slot, first head, count) of every run of consecutive heads
+            out, i = [], 0
+            while i < len(heads):
+                j = i
+                while j + 1 < len(heads) and heads[j + 1] == heads[j] + 1:
+                    j += 1
+                out.append((s0 + i, heads[i], j - i + 1))
+                i = j + 1
+            return out
+
+        for (s0, s1, sub, heads) in groups:
             with torch.cuda.stream(s_in):
-                for dev, host in ((q_dev, q_host), (k_dev, k_host), (v_dev, v_host)):
-                    dev[:, h0:h1].copy_(host[:, h0:h1], non_blocking=True)
+                for (sl, h, n) in runs(s0, heads):
+                    for dev, host in ((q_dev, q_host), (k_dev, k_host), (v_dev, v_host)):
+                        dev[:, sl:sl + n].copy_(host[:, h:h + n], non_blocking=True)
                 arrived = torch.cuda.Event()
                 arrived.record(s_in)
             s_cmp.wait_event(arrived)
             with torch.cuda.stream(s_cmp):
-                sub.forward(q_dev[:, h0:h1], k_dev[:, h0:h1], v_dev[:, h0:h1], method,
-                            list(budgets)[h0:h1], keep_k, dense_q, rounds, rho, eps, seed,
+                sub.forward(q_dev[:, s0:s1], k_dev[:, s0:s1], v_dev[:, s0:s1], method,
+                            [budgets[h] for h in heads], keep_k, dense_q, rounds, rho, eps, seed,
                             stream=s_cmp, top_p=top_p)
                 done = torch.cuda.Event()
                 done.record(s_cmp)
             s_out.wait_event(done)
             with torch.cuda.stream(s_out):
-                out_host[:, h0:h1].copy_(sub.out, non_blocking=True)
+                for (sl, h, n) in runs(0, heads):
+                    out_host[:, h:h + n].copy_(sub.out[:, sl:sl + n], non_blocking=True)
         for s in (s_in, s_cmp, s_out):
             main.wait_stream(s)
         return out_host

@@ -424,12 +424,15 @@ def test_schedule_many_rows_and_repeated_counts():
     assert order.cpu().tolist() == sorted(range(384), key=lambda it: (-flat[it], it))
 
 
-@pytest.mark.parametrize("method", ["mass", "drift"])
-def test_host_buffer_path_in_head_groups_equals_forward(method):
+@pytest.mark.parametrize("method,planned", [("mass", False), ("drift", False), ("drift", True)])
+def test_host_buffer_path_in_head_groups_equals_forward(method, planned):
     """forward_host (pinned host tensors, heads in groups on overlapping streams) gives the
-    same bytes as forward() on device tensors: every step is per head."""
+    same bytes as forward() on device tensors: every step is per head.  `planned`: the
+    heads are regrouped by budget (plan_head_order), so the staging slots are permuted."""
     ensure_built()
     wl = W.make_workload(2, heads=4, views=6, method=method, sparsity=0.75, rounds=3)
+    if planned:
+        wl.budgets = [wl.budgets[0] // 3, wl.budgets[1], wl.budgets[2] // 2, wl.budgets[3] * 2]
     dev = torch.device("cuda")
     B, H, N, _ = wl.q.shape
     ref = SparseGlobalAttention(B, H, N, device=dev)
@@ -437,7 +440,9 @@ def test_host_buffer_path_in_head_groups_equals_forward(method):
     ref.forward(wl.q.to(dev), wl.k.to(dev), wl.v.to(dev), METHODS[method], wl.budgets,
                 wl.keep_k.to(dev), wl.dense_q.to(dev), wl.rounds, wl.rho, wl.eps, wl.select_seed)
     layer = SparseGlobalAttention(B, H, N, device=dev)
-    layer.make_groups(wl.w_o.to(dev), 3)
+    layer.make_groups(wl.w_o.to(dev), 3, budgets=wl.budgets if planned else None)
+    if planned:
+        assert layer._order != list(range(H))
     qh, kh, vh = (t.cpu().pin_memory() for t in (wl.q, wl.k, wl.v))
     outh = torch.empty(B, H, N, 64, dtype=torch.bfloat16).pin_memory()
     for _ in range(2):

@@ -90,3 +90,24 @@ def test_host_path_head_group_sizes():
                     assert max(sizes) - min(sizes) <= 1
     assert S.group_sizes(16, 4, taper=True) == [6, 5, 3, 2]
     assert S.group_sizes(16, 6) == [3, 3, 3, 3, 2, 2]
+
+
+def test_host_path_head_order_by_budget():
+    """plan_head_order: a permutation of the heads; the last group holds the cheapest
+    heads; the other groups' work per head is balanced (largest first to the least loaded
+    group per head); identity with one group; ascending within each group."""
+    from block_sparse_global_b200.pipeline import SparseGlobalAttention as S
+    budgets = [142, 80, 226, 14, 104, 207, 58, 58, 85, 123, 25, 74, 52, 254, 135, 75]
+    sizes = S.group_sizes(16, 6)
+    order = S.plan_head_order(budgets, sizes)
+    assert sorted(order) == list(range(16))
+    assert sorted(order[-sizes[-1]:]) == sorted(sorted(range(16), key=lambda h: (budgets[h], h))[:sizes[-1]])
+    groups, s0 = [], 0
+    for n in sizes:
+        groups.append(order[s0:s0 + n])
+        s0 += n
+    assert all(g == sorted(g) for g in groups)
+    per_head = [sum(budgets[h] + 16 for h in g) / len(g) for g in groups[:-1]]
+    assert max(per_head) - min(per_head) <= max(budgets) / 3, per_head
+    assert S.plan_head_order(budgets, [16]) == list(range(16))
+    assert S.plan_head_order([5, 5, 5, 5], [2, 2]) == [2, 3, 0, 1]
