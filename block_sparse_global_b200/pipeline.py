@@ -246,7 +246,8 @@ class SparseGlobalAttention:
             sub.load_output_projection(w_o[:, cols])
             self._groups.append((s0, s0 + n, sub, heads))
             s0 += n
-        self._streams = [torch.cuda.Stream(self.device) for _ in range(3)]
+        # copies in, kernels of even groups, copies out, kernels of odd groups
+        self._streams = [torch.cuda.Stream(self.device) for _ in range(4)]
         return self._groups
 
     def forward_host(self, q_host, k_host, v_host, out_host, method: int, budgets: Sequence[int],
@@ -255,8 +256,10 @@ class SparseGlobalAttention:
                      top_p: float = 1.0):
         """The layer end to end from pinned host tensors [1,H,N,64] bf16 to the pinned host
         output.  Heads are processed in the groups of make_groups(): the copy in of group
-        g+1, the kernels of group g and the copy out of group g-1 run on three streams and
-        overlap.  The device staging tensors hold the heads in processing order (slot s
+        g+1, the kernels of group g and the copy out of group g-1 overlap, and the kernels
+        of consecutive groups run on two streams (every group has its own buffers), so that
+        a group's selection can fill the SMs that the previous group's attention leaves
+        idle in its last wave.  The device staging tensors hold the heads in processing order (slot s
         holds head make_groups' order[s]); contiguous runs of heads are copied in one piece.
         RANDOM selection runs as one group in head order (its keys depend on the head index
         within the call).  The caller's current stream waits for the whole layer.
@@ -270,9 +273,9 @@ class SparseGlobalAttention:
         k_dev = torch.empty_like(k_host, device=self.device) if k_dev is None else k_dev
         v_dev = torch.empty_like(v_host, device=self.device) if v_dev is None else v_dev
         budgets = list(budgets)
-        s_in, s_cmp, s_out = self._streams
+        s_in, s_even, s_out, s_odd = self._streams
         main = torch.cuda.current_stream(self.device)
-        for s in (s_in, s_cmp, s_out):
+        for s in self._streams:
             s.wait_stream(main)
 
         def runs(s0, heads):
@@ -286,7 +289,8 @@ class SparseGlobalAttention:
                 i = j + 1
             return out
 
-        for (s0, s1, sub, heads) in groups:
+        for gi, (s0, s1, sub, heads) in enumerate(groups):
+            s_cmp = s_odd if gi % 2 else s_even
             with torch.cuda.stream(s_in):
                 for (sl, h, n) in runs(s0, heads):
                     for dev, host in ((q_dev, q_host), (k_dev, k_host), (v_dev, v_host)):
@@ -304,7 +308,7 @@ class SparseGlobalAttention:
             with torch.cuda.stream(s_out):
                 for (sl, h, n) in runs(0, heads):
                     out_host[:, h:h + n].copy_(sub.out[:, sl:sl + n], non_blocking=True)
-        for s in (s_in, s_cmp, s_out):
+        for s in self._streams:
             main.wait_stream(s)
         return out_host
 
