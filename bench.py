@@ -66,8 +66,9 @@ def parse():
                          "to HBM before the step instead of during its first kernel's reads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--e2e-groups", type=int, default=6,
-                    help="head groups of the host-buffer call (copy in / kernels / copy out overlap)")
+    ap.add_argument("--e2e-groups", type=int, default=None,
+                    help="head groups of the host-buffer call (copy in / kernels / copy out overlap); "
+                         "default: 9 when a head's Q, K and V take at least 32 MB, else 6")
     ap.add_argument("--e2e-split", default=None,
                     help="explicit heads per group of the host-buffer call, e.g. 8,4,2,1,1")
     ap.add_argument("--e2e-taper", action="store_true",
@@ -484,7 +485,12 @@ def run_ours(args):
             outh = torch.empty(layer.out.shape, dtype=layer.out.dtype).pin_memory()
             qd, kd, vd = (torch.empty_like(x) for x in (q, k, v))
             # head groups: copies in, kernels and copies out overlap on three streams
-            groups = 1 if wl.method == R.SELECT_RANDOM else max(1, min(args.e2e_groups, H))
+            # more, smaller groups once a head's copy is long enough that the per-copy
+            # overhead no longer shows (the 100-view layer); the kernels of consecutive
+            # groups overlap on two streams
+            per_head = 3 * q[0, 0].numel() * q.element_size()
+            want = args.e2e_groups if args.e2e_groups else (9 if per_head >= 32 << 20 else 6)
+            groups = 1 if wl.method == R.SELECT_RANDOM else max(1, min(want, H))
             split = [int(x) for x in args.e2e_split.split(",")] if args.e2e_split else None
             layer.make_groups(wl.w_o, groups, taper=args.e2e_taper,
                               sizes=split if wl.method != R.SELECT_RANDOM else None,

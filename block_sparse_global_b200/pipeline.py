@@ -200,10 +200,11 @@ class SparseGlobalAttention:
         left after the last copy in), and the other heads are spread over the other groups
         largest first, each to the group with the least work per head so far, so that no
         group's kernels outlast the next group's copy in.  Heads keep ascending order
-        within a group."""
+        within a group.  With equal budgets the heads stay in order (contiguous heads are
+        copied in one piece)."""
         H, G = len(budgets), len(sizes)
-        if G <= 1:
-            return list(range(H))
+        if G <= 1 or len(set(int(b) for b in budgets)) == 1:
+            return list(range(H))  # equal budgets: nothing to balance, keep the copies whole
         cost = [int(b) + 16 for b in budgets]  # kept candidates + always-kept / fixed work
         asc = sorted(range(H), key=lambda h: (cost[h], h))
         last = asc[:sizes[-1]]

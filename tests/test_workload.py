@@ -110,4 +110,5 @@ def test_host_path_head_order_by_budget():
     per_head = [sum(budgets[h] + 16 for h in g) / len(g) for g in groups[:-1]]
     assert max(per_head) - min(per_head) <= max(budgets) / 3, per_head
     assert S.plan_head_order(budgets, [16]) == list(range(16))
-    assert S.plan_head_order([5, 5, 5, 5], [2, 2]) == [2, 3, 0, 1]
+    assert S.plan_head_order([5, 5, 5, 5], [2, 2]) == [0, 1, 2, 3]
+    assert S.plan_head_order([5, 5, 5, 6], [2, 2]) == [2, 3, 0, 1]
