@@ -112,3 +112,48 @@ def test_host_path_head_order_by_budget():
     assert S.plan_head_order(budgets, [16]) == list(range(16))
     assert S.plan_head_order([5, 5, 5, 5], [2, 2]) == [0, 1, 2, 3]
     assert S.plan_head_order([5, 5, 5, 6], [2, 2]) == [2, 3, 0, 1]
+
+
+def test_host_path_group_plan_rejects_bad_input_and_maps_every_head():
+    """make_groups: sizes must cover the heads, budgets must name every head; the planned
+    groups' slots and heads form a bijection and each group's W_O columns are its heads'."""
+    import pytest
+    import torch
+    from block_sparse_global_b200.pipeline import SparseGlobalAttention as S
+    layer = S.__new__(S)  # host-side planning only: no device buffers
+    layer.B, layer.H, layer.N, layer.key_block = 1, 6, 256, 128
+    layer.device = torch.device("cpu")
+    calls = []
+
+    class _Sub:
+        def __init__(self, B, H, N, device=None, key_block=128):
+            self.H = H
+
+        def load_output_projection(self, w):
+            calls.append(w)
+
+    import block_sparse_global_b200.pipeline as P
+    real, P.SparseGlobalAttention = P.SparseGlobalAttention, _Sub
+    real_stream = torch.cuda.Stream
+    torch.cuda.Stream = lambda *a, **k: None
+    try:
+        w_o = torch.arange(64 * 6, dtype=torch.float32).repeat(3, 1)  # column c holds c
+        with pytest.raises(ValueError):
+            S.make_groups(layer, w_o, 2, sizes=[3, 2])
+        with pytest.raises(ValueError):
+            S.make_groups(layer, w_o, 2, sizes=[6, 0])
+        with pytest.raises(ValueError):
+            S.make_groups(layer, w_o, 2, budgets=[1, 2, 3])  # not one budget per head
+        groups = S.make_groups(layer, w_o, 3, budgets=[9, 1, 5, 7, 2, 8])
+    finally:
+        P.SparseGlobalAttention = real
+        torch.cuda.Stream = real_stream
+    slots, heads = [], []
+    for (s0, s1, sub, hs), w in zip(groups, calls[-len(groups):]):
+        assert s1 - s0 == len(hs) == sub.H
+        slots += list(range(s0, s1))
+        heads += hs
+        want = torch.cat([torch.arange(64 * h, 64 * h + 64, dtype=torch.float32) for h in hs])
+        assert torch.equal(w[0], want)
+    assert slots == list(range(6)) and sorted(heads) == list(range(6))
+    assert groups[-1][3] == sorted([1, 4])  # the two cheapest heads last
